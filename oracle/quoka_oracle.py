@@ -1,0 +1,247 @@
+"""fp64 CPU oracle for QUOKA-style KV selection followed by sparse chunk attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import or call this
+module; only the tests, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` use it.  It shares no code with the CUDA
+library and imports nothing from the product package.
+
+What it computes, and where each step comes from
+------------------------------------------------
+Sources are the QUOKA page ("Qualcomm QuoKA: ... 5x", arXiv 2602.08722), its
+method summary and the captions of Figure 1 and Figure 2, plus the multi-query
+attention page ("Multi-Query Attention", technical insight section) for the
+sharing of one K/V head by several query heads.
+
+QUOKA is a heuristic selection followed by exact dense attention over the selected
+set, so the oracle follows the method's steps in the pages' order:
+
+1. mean query (method summary; Q&A 1): per query head, the mean of the chunk's
+   unit-normalised queries, m = (1/C) sum_t q_t / |q_t|.
+2. query subselection (Figure 1(b): "filter queries by cosine dissimilarity";
+   Figure 2: queries with high S_q interact more strongly): c_t = cos(q_t, m);
+   keep the Nq queries with the smallest c_t (largest S_q = -c_t); ties go to
+   the lower chunk position.  Nq >= C keeps every query.
+3. cosine scoring (Figure 1(b): "query-key cosine similarity filters keys"):
+   cos(q_i, k_j) for every kept query i and every prefix key j < P.
+4. group-aware aggregation (method summary: max pooling "to preserve important
+   interactions", mean pooling "to adapt to GQA", respectively): per key, max over
+   the kept queries of each query head, then mean over the G heads sharing the
+   KV head.
+5. top-B (Figure 1(a): the KV cache is sub-selected into a "compacted cache"):
+   per KV head the B best-scoring prefix keys, ties to the lower cache index,
+   returned in ascending index order; P <= B keeps every prefix key.
+6. dense attention over the compacted cache (Figure 1(a)): query t of head h
+   attends to the selected prefix keys of KV head h // G plus the chunk's own
+   keys P .. P+t (causal), softmax(q k^T / sqrt(d)) v.
+
+Readings where the pages are silent (each is listed with its reason in the design
+notes of the repository): the budget B counts prefix keys only and the chunk's own
+causal keys are always attended; the mean query is per query head and over
+*normalised* queries; a zero vector has cosine 0 with everything; the softmax scale
+is 1/sqrt(d); head h maps to KV head h // G.
+
+All arithmetic is float64 on exact copies of the (fp32 or bf16) inputs.
+Pins: tests/test_oracle.py checks every step against brute force, closed forms,
+invariants and an independent library routine.  End-to-end agreement with the
+authors' own implementation is "parity unpinned": the pages print no worked numbers.
+"""
+from __future__ import annotations
+
+from typing import Dict, Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "unit_rows", "mean_query", "query_cosines", "subselect_queries", "pooled_key_scores",
+    "top_budget", "select_chunk", "attend_chunk", "select_batch", "attend_batch",
+]
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):                       # a torch tensor: exact widening
+        x = x.detach().to("cpu")
+        import torch  # local: only for the dtype conversion of torch inputs
+        x = x.to(torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def unit_rows(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Row norms and unit rows of x [n, d]; a zero row stays zero (cosine 0)."""
+    x = _f64(x)
+    n = np.sqrt(np.einsum("nd,nd->n", x, x))
+    u = np.zeros_like(x)
+    nz = n > 0
+    u[nz] = x[nz] / n[nz, None]
+    return n, u
+
+
+def mean_query(q: np.ndarray, raw: bool = False) -> np.ndarray:
+    """Step 1: the chunk's mean query for one head, q [C, d] -> [d].
+
+    ``raw=True`` averages the unnormalised queries instead; it exists only so the
+    tests can show that this alternative reading breaks the per-query scale
+    invariance that the cosine-based method has.
+    """
+    q = _f64(q)
+    if raw:
+        return q.mean(axis=0)
+    _, u = unit_rows(q)
+    return u.mean(axis=0)
+
+
+def query_cosines(q: np.ndarray, raw_mean: bool = False) -> np.ndarray:
+    """Step 2a: c_t = cos(q_t, m) for one head, q [C, d] -> [C]."""
+    _, u = unit_rows(q)
+    m = mean_query(q, raw=raw_mean)
+    mn = np.sqrt(m @ m)
+    if mn == 0.0:
+        return np.zeros(u.shape[0])
+    return u @ (m / mn)
+
+
+def subselect_queries(q: np.ndarray, nq: int, raw_mean: bool = False) -> np.ndarray:
+    """Step 2b: indices (ascending) of the min(nq, C) queries least similar to the mean.
+
+    Ordering key: cosine ascending, then chunk position ascending.
+    """
+    c = query_cosines(q, raw_mean=raw_mean)
+    C = c.shape[0]
+    if nq >= C:
+        return np.arange(C, dtype=np.int64)
+    order = np.lexsort((np.arange(C), c))
+    return np.sort(order[:nq]).astype(np.int64)
+
+
+def pooled_key_scores(kept_units: Sequence[np.ndarray], k: np.ndarray,
+                      block: int = 8192) -> np.ndarray:
+    """Steps 3-4 for one KV head.
+
+    kept_units: one array [Nk_h, d] of unit kept queries per query head of the group.
+    k: prefix keys [P, d].  Returns score [P]:
+        score_j = mean_h max_{i in K_h} (u_i . k_j) / |k_j|   (0 for a zero key).
+    Keys are processed in blocks only to bound memory; no reordering of the
+    arithmetic beyond that.
+    """
+    k = _f64(k)
+    P = k.shape[0]
+    out = np.zeros(P)
+    if P == 0:
+        return out
+    G = len(kept_units)
+    for s in range(0, P, block):
+        kb = k[s:s + block]
+        r, _ = unit_rows(kb)
+        acc = np.zeros(kb.shape[0])
+        for uh in kept_units:
+            dots = _f64(uh) @ kb.T                      # [Nk_h, blk]
+            acc += dots.max(axis=0)
+        acc /= G
+        nz = r > 0
+        blk = np.zeros(kb.shape[0])
+        blk[nz] = acc[nz] / r[nz]
+        out[s:s + block] = blk
+    return out
+
+
+def top_budget(score: np.ndarray, budget: int) -> np.ndarray:
+    """Step 5: the min(budget, P) best prefix keys, ties to the lower index, ascending."""
+    score = _f64(score)
+    P = score.shape[0]
+    if budget >= P:
+        return np.arange(P, dtype=np.int64)
+    order = np.lexsort((np.arange(P), -score))
+    return np.sort(order[:budget]).astype(np.int64)
+
+
+def select_chunk(q_chunk, k_seq, prefix_len: int, nq: int, budget: int,
+                 kept_override: Optional[Sequence[np.ndarray]] = None,
+                 raw_mean: bool = False) -> Dict[str, object]:
+    """Steps 1-5 for one sequence.
+
+    q_chunk [H_q, C, d]; k_seq [H_kv, >= P, d] (rows of this sequence only).
+    ``kept_override`` replaces step 2's kept sets (one index array per query head),
+    used to re-score with another implementation's kept sets when those differ only
+    by near-ties.
+    Returns kept (list per query head), cos [H_q, C], score [H_kv, P], idx (list per
+    KV head, ascending).
+    """
+    q = _f64(q_chunk)
+    H_q, C, d = q.shape
+    k = _f64(k_seq)
+    H_kv = k.shape[0]
+    G = H_q // H_kv
+    P = int(prefix_len)
+    cos = np.stack([query_cosines(q[h], raw_mean=raw_mean) for h in range(H_q)]) if C else \
+        np.zeros((H_q, 0))
+    if kept_override is not None:
+        kept = [np.sort(np.asarray(x, dtype=np.int64)) for x in kept_override]
+    else:
+        kept = [subselect_queries(q[h], nq, raw_mean=raw_mean) for h in range(H_q)]
+    score = np.zeros((H_kv, P))
+    idx: List[np.ndarray] = []
+    for g in range(H_kv):
+        units = []
+        for h in range(g * G, (g + 1) * G):
+            _, u = unit_rows(q[h])
+            units.append(u[kept[h]])
+        score[g] = pooled_key_scores(units, k[g, :P])
+        idx.append(top_budget(score[g], budget))
+    return {"kept": kept, "cos": cos, "score": score, "idx": idx}
+
+
+def attend_chunk(q_chunk, k_seq, v_seq, prefix_len: int, idx: Sequence[np.ndarray],
+                 rows: Optional[Iterable[Tuple[int, int]]] = None) -> np.ndarray:
+    """Step 6 for one sequence.
+
+    q_chunk [H_q, C, d]; k_seq, v_seq [H_kv, >= P + C, d]; idx: per KV head the
+    selected prefix indices.  Returns O [H_q, C, d], or, when ``rows`` is given, an
+    array [len(rows), d] holding only those (head, position) rows.
+    """
+    q = _f64(q_chunk)
+    H_q, C, d = q.shape
+    k = _f64(k_seq)
+    v = _f64(v_seq)
+    H_kv = k.shape[0]
+    G = H_q // H_kv
+    P = int(prefix_len)
+    scale = 1.0 / np.sqrt(d)
+    want = None if rows is None else list(rows)
+    heads = range(H_q) if want is None else sorted({h for h, _ in want})
+    out = {}
+    for h in heads:
+        g = h // G
+        sel = np.asarray(idx[g], dtype=np.int64)
+        sel = sel[sel >= 0]
+        ks = np.concatenate([k[g, sel], k[g, P:P + C]], axis=0)
+        vs = np.concatenate([v[g, sel], v[g, P:P + C]], axis=0)
+        ns = sel.shape[0]
+        ts = range(C) if want is None else sorted({t for hh, t in want if hh == h})
+        for t in ts:
+            n_keys = ns + t + 1                        # selected prefix + chunk keys P..P+t
+            logits = (ks[:n_keys] @ q[h, t]) * scale
+            mx = logits.max()
+            p = np.exp(logits - mx)
+            out[(h, t)] = (p @ vs[:n_keys]) / p.sum()
+    if want is None:
+        o = np.zeros((H_q, C, d))
+        for (h, t), val in out.items():
+            o[h, t] = val
+        return o
+    return np.stack([out[r] for r in want]) if want else np.zeros((0, d))
+
+
+def _seq_rows(x, kv_off, b):
+    return x[:, kv_off[b]:kv_off[b + 1]]
+
+
+def select_batch(q, k_cache, kv_off, prefix_len, nq, budget):
+    """select_chunk over a batch: q [batch, H_q, C, d], k_cache [H_kv, total, d]."""
+    return [select_chunk(q[b], _seq_rows(k_cache, kv_off, b), prefix_len[b], nq, budget[b])
+            for b in range(len(prefix_len))]
+
+
+def attend_batch(q, k_cache, v_cache, kv_off, prefix_len, idx_per_seq):
+    """attend_chunk over a batch; idx_per_seq[b] is a list of per-KV-head index arrays."""
+    return np.stack([attend_chunk(q[b], _seq_rows(k_cache, kv_off, b),
+                                  _seq_rows(v_cache, kv_off, b), prefix_len[b], idx_per_seq[b])
+                     for b in range(len(prefix_len))])

@@ -1,0 +1,182 @@
+"""Seeded synthetic workloads for one chunk of a chunked prefill.
+
+This module only *draws* tensors: it holds none of the selection or attention
+arithmetic, so both the CUDA path (through the binding) and the fp64 oracle can be
+fed from it without sharing any method code.
+
+Five workloads are defined, matching the shapes of the QUOKA page's chunked-prefill
+setting (page "Qualcomm QuoKA ...", Figure 1(a): a prompt split into chunks, each
+chunk attending over a compacted KV cache) and its ~12 % KV budget (same page,
+results section):
+
+    tiny_mqa      H_q=4, H_kv=1, d=64, prompt 512 in 4 chunks of 128, Nq=16, B=128, fp32
+    gqa_8k        H_q=32, H_kv=8, d=128, prefix 8192 + chunk 512, Nq=64, B=1024, bf16
+    long_chunk    H_q=64, H_kv=8, d=128, prefix 32768 + chunk 2048, Nq=128, B=4096, bf16
+    ctx_128k      H_q=32, H_kv=8, d=128, prefix 131072 + chunk 4096, Nq=128, B=16384, bf16
+    ragged_8      8 sequences, prefix ~ U[4096, 65536], chunk 1024, H_q=64, H_kv=4,
+                  d=128, Nq=64, B = 12 % of each prefix rounded to 64, bf16
+
+Value recipes (all drawn in fp32 from ``torch.Generator('cpu').manual_seed(seed)``
+and then rounded once to the workload dtype):
+
+    gauss   Q, K, V ~ N(0, 1)
+    rank4   Q, K ~ N(0, 1) + 2 * U_g z, with U_g an orthonormal d x 4 basis per KV
+            head (QR of a Gaussian) and z ~ N(0, I_4) per token and head; V ~ N(0, 1)
+    heavy   N(0, 1), then per (sequence, KV head) 2 % of the prefix rows (without
+            replacement) are replaced by 3 * sqrt(d) * q_hat, q_hat the direction of a
+            uniformly drawn chunk query of a uniformly drawn head of that group
+
+KV cache layout: ``k_cache``/``v_cache`` are [H_kv, kv_total, d]; sequence b owns rows
+``[kv_off[b], kv_off[b+1])`` holding its prefix followed by its own chunk rows.
+Queries are [batch, H_q, C, d].
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Tuple
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    h_q: int
+    h_kv: int
+    head_dim: int
+    chunk: int
+    prefix: Tuple[int, ...]          # per sequence (for prompt workloads: chunk 0's)
+    nq: int
+    budget: Tuple[int, ...]          # per sequence, counts prefix keys only
+    dtype: str                       # "f32" or "bf16"
+    seed: int
+    recipe: str                      # "gauss", "rank4" or "heavy"
+    prompt_chunks: int = 1           # >1: whole prompt of prompt_chunks * chunk tokens
+
+    @property
+    def batch(self) -> int:
+        return len(self.prefix)
+
+    @property
+    def group(self) -> int:
+        return self.h_q // self.h_kv
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def elem_bytes(self) -> int:
+        return 4 if self.dtype == "f32" else 2
+
+    def seq_rows(self) -> Tuple[int, ...]:
+        """Rows each sequence owns in the cache (prefix plus every chunk it will run)."""
+        return tuple(p + self.chunk * self.prompt_chunks for p in self.prefix)
+
+    def chunk_steps(self):
+        """(chunk index, per-sequence prefix lengths) for every chunk step of the workload."""
+        for c in range(self.prompt_chunks):
+            yield c, tuple(p + c * self.chunk for p in self.prefix)
+
+
+def _budget_12pct(p: int) -> int:
+    """12 % of a prefix, rounded to a multiple of 64 (halves up), at least 64."""
+    return max(64, 64 * int(math.floor(0.12 * p / 64.0 + 0.5)))
+
+
+def _ragged_prefixes(seed: int) -> Tuple[int, ...]:
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return tuple(int(x) for x in torch.randint(4096, 65537, (8,), generator=g))
+
+
+_RAGGED = _ragged_prefixes(4)
+
+WORKLOADS: Dict[str, Workload] = {
+    "tiny_mqa": Workload("tiny_mqa", 4, 1, 64, 128, (0,), 16, (128,), "f32", 0, "gauss",
+                         prompt_chunks=4),
+    "gqa_8k": Workload("gqa_8k", 32, 8, 128, 512, (8192,), 64, (1024,), "bf16", 1, "rank4"),
+    "long_chunk": Workload("long_chunk", 64, 8, 128, 2048, (32768,), 128, (4096,), "bf16", 2,
+                           "heavy"),
+    "ctx_128k": Workload("ctx_128k", 32, 8, 128, 4096, (131072,), 128, (16384,), "bf16", 3,
+                         "heavy"),
+    "ragged_8": Workload("ragged_8", 64, 4, 128, 1024, _RAGGED, 64,
+                         tuple(_budget_12pct(p) for p in _RAGGED), "bf16", 4, "rank4"),
+}
+
+# The headline single-GPU workload (128K context).
+HEADLINE = "ctx_128k"
+
+
+def custom(name: str = "custom", *, h_q: int, h_kv: int, head_dim: int, chunk: int,
+           prefix, nq: int, budget, dtype: str = "bf16", seed: int = 0,
+           recipe: str = "gauss", prompt_chunks: int = 1) -> Workload:
+    """A small ad-hoc workload (tests use these for edge cases)."""
+    prefix = tuple(int(p) for p in (prefix if hasattr(prefix, "__len__") else (prefix,)))
+    if not hasattr(budget, "__len__"):
+        budget = (int(budget),) * len(prefix)
+    return Workload(name, h_q, h_kv, head_dim, chunk, prefix, nq, tuple(int(b) for b in budget),
+                    dtype, seed, recipe, prompt_chunks)
+
+
+@dataclasses.dataclass
+class Tensors:
+    """CPU tensors of one workload, already rounded to the workload dtype."""
+    q: torch.Tensor          # [batch, H_q, prompt_chunks * C, d]
+    k_cache: torch.Tensor    # [H_kv, kv_total, d]
+    v_cache: torch.Tensor    # [H_kv, kv_total, d]
+    kv_off: Tuple[int, ...]  # batch + 1 row offsets
+
+    def q_chunk(self, c: int, chunk: int) -> torch.Tensor:
+        return self.q[:, :, c * chunk:(c + 1) * chunk, :].contiguous()
+
+
+def _orthonormal(g: torch.Generator, d: int, r: int) -> torch.Tensor:
+    a = torch.randn(d, r, generator=g, dtype=torch.float64)
+    qmat, _ = torch.linalg.qr(a)
+    return qmat.to(torch.float32)
+
+
+def generate(w: Workload) -> Tensors:
+    """Draw the workload's Q and KV cache on the CPU from its seed."""
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    d = w.head_dim
+    rows = w.seq_rows()
+    kv_off = [0]
+    for r in rows:
+        kv_off.append(kv_off[-1] + r)
+    total = kv_off[-1]
+    qlen = w.chunk * w.prompt_chunks
+
+    q = torch.randn(w.batch, w.h_q, qlen, d, generator=g)
+    k = torch.randn(w.h_kv, total, d, generator=g)
+    v = torch.randn(w.h_kv, total, d, generator=g)
+
+    if w.recipe == "rank4":
+        for kv in range(w.h_kv):
+            basis = _orthonormal(g, d, 4)                               # [d, 4]
+            zk = torch.randn(total, 4, generator=g)
+            k[kv] += 2.0 * zk @ basis.T
+            for h in range(kv * w.group, (kv + 1) * w.group):
+                zq = torch.randn(w.batch, qlen, 4, generator=g)
+                q[:, h] += 2.0 * zq @ basis.T
+    elif w.recipe == "heavy":
+        scale = 3.0 * math.sqrt(d)
+        for b in range(w.batch):
+            p = w.prefix[b]
+            n_heavy = int(round(0.02 * p))
+            if n_heavy == 0:
+                continue
+            for kv in range(w.h_kv):
+                pos = torch.randperm(p, generator=g)[:n_heavy]
+                heads = torch.randint(kv * w.group, (kv + 1) * w.group, (n_heavy,), generator=g)
+                toks = torch.randint(0, qlen, (n_heavy,), generator=g)
+                src = q[b, heads, toks]                                  # [n_heavy, d]
+                src = src / src.norm(dim=-1, keepdim=True).clamp_min(1e-30)
+                k[kv, kv_off[b] + pos] = scale * src
+    elif w.recipe != "gauss":
+        raise ValueError(f"unknown recipe {w.recipe!r}")
+
+    dt = w.torch_dtype
+    return Tensors(q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous(),
+                   tuple(kv_off))
