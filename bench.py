@@ -1,0 +1,377 @@
+"""Throughput of one chunked-prefill step (QUOKA selection + sparse chunk attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input: the
+select call (query subselect, cosine scoring + pooling, top-B) and the attention
+call, through the C ABI.  Default workload: the 128K-context chunk (prefix 131072 +
+chunk 4096, H_q 32, H_kv 8, d 128, Nq 128, B 16384, bf16).  Each timed step is
+bracketed by CUDA events on the launching stream, with a 256 MB L2 flush before it
+(outside the events).  Under torchrun every rank runs its own independent chunk step
+(weak scaling, no collective on the data path) and the slowest rank's time is used.
+
+Rank 0 prints one JSON line.  `--impl reference` times the fp64 CPU oracle instead
+(test infrastructure, run on the host cores on a bounded sample of the workload).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from query_oriented_sparse_b200 import workloads as W  # noqa: E402
+
+METRIC = "chunked-prefill sparse-attn tokens/s (select+attend) and % of roofline, 1 B200"
+UNIT = "tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 4  # qsub, score, top-k, attention
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def stage_model(w: W.Workload):
+    """Algorithmic bytes and FLOPs per stage for one chunk step (compulsory traffic:
+    the selection reads every prefix key once; attention reads only the selected and
+    causal keys; tile padding and the 4-byte pooled intermediate are not counted)."""
+    s, d, C, nq = w.elem_bytes, w.head_dim, w.chunk, min(w.nq, w.chunk)
+    st = {k: {"bytes": 0.0, "flops": 0.0} for k in ("qsub", "score", "topk", "attn")}
+    for P, B in zip(w.prefix, w.budget):
+        n = min(B, P)
+        st["qsub"]["bytes"] += w.h_q * C * d * s + w.h_q * nq * d * s
+        st["score"]["bytes"] += w.h_kv * P * d * s + w.h_q * nq * d * s
+        st["score"]["flops"] += 2.0 * w.h_q * nq * P * d
+        st["topk"]["bytes"] += w.h_kv * n * 4
+        st["attn"]["bytes"] += (2 * w.h_q * C * d * s + 2 * w.h_kv * (n + C) * d * s +
+                                w.h_kv * n * 4)
+        st["attn"]["flops"] += 4.0 * d * w.h_q * (C * n + C * (C + 1) / 2)
+    return st
+
+
+def roofline_us(st, peaks):
+    out = {}
+    for k, v in st.items():
+        out[k] = max(v["flops"] / (peaks["bf16_tflops"] * 1e12),
+                     v["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e6
+    return out
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.sel = str(device_index)
+        try:
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            self.sel = "GPU-" + str(uuid)
+        except Exception:
+            pass
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", self.sel, "-lms", "200"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------------------
+# CPU oracle arm
+# --------------------------------------------------------------------------------------
+
+def oracle_sample(w: W.Workload, t: W.Tensors, rows: int = 64):
+    """Times the fp64 oracle on a bounded sample of one chunk step: the complete
+    selection of KV head 0 of sequence 0 plus attention for `rows` query rows of its
+    group; extrapolates to the whole step (all KV heads and query rows, all sequences)."""
+    from oracle import quoka_oracle as O
+    b, g = 0, 0
+    P, B = w.prefix[b], w.budget[b]
+    lo, hi = t.kv_off[b], t.kv_off[b + 1]
+    G = w.group
+    q = t.q_chunk(0, w.chunk)[b, g * G:(g + 1) * G].double().numpy()
+    k = t.k_cache[g:g + 1, lo:hi].double().numpy()
+    v = t.v_cache[g:g + 1, lo:hi].double().numpy()
+    t0 = time.perf_counter()
+    res = O.select_chunk(q, k, P, w.nq, B)
+    t_sel = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    rr = [(int(rng.integers(G)), int(rng.integers(w.chunk))) for _ in range(rows)]
+    t0 = time.perf_counter()
+    O.attend_chunk(q, k, v, P, res["idx"], rows=rr)
+    t_att = time.perf_counter() - t0
+    # the sampled sequence stands for the others in proportion to their prefix
+    scale_sel = sum(w.prefix) / max(P, 1) if P else w.batch
+    est = t_sel * w.h_kv * scale_sel + t_att / rows * (w.h_q * w.chunk * w.batch)
+    return {"t_select_s": t_sel, "t_attn_s": t_att, "est_step_s": est,
+            "tokens_per_s": w.batch * w.chunk / est,
+            "sample": f"selection of KV head 0 of sequence 0 (P={P}) + attention for {rows} "
+                      f"sampled query rows of its group; extrapolated to {w.h_kv} KV heads x "
+                      f"{w.h_q * w.chunk * w.batch} query rows"}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    t = W.generate(w)
+    samples = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(w, t)
+        if i >= args.warmup:
+            samples.append(r)
+    v = statistics.median(s["tokens_per_s"] for s in samples)
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * w.batch * w.chunk / v, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "chunk": w.chunk,
+                   "prefix": list(w.prefix), "h_q": w.h_q, "h_kv": w.h_kv, "head_dim": w.head_dim,
+                   "nq": w.nq, "budget": list(w.budget), "input_dtype": w.dtype},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": samples[0]["sample"]},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------------------
+
+def run_ours(args, w):
+    from query_oriented_sparse_b200 import binding as Bd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    peaks, peak_src = load_peaks()
+
+    t = W.generate(w)
+    q = t.q.to(dev)
+    k = t.k_cache.to(dev)
+    v = t.v_cache.to(dev)
+    shape = Bd.shape_of(q, k)
+    b_max = max(w.budget)
+    ws = torch.empty(Bd.select_workspace_size(shape, max(w.prefix), w.nq), dtype=torch.uint8,
+                     device=dev)
+    idx = torch.empty(w.batch, w.h_kv, b_max, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        Bd.quoka_select(q, k, t.kv_off, w.prefix, w.nq, w.budget, b_max, idx_out=idx,
+                        workspace=ws)
+        Bd.sparse_chunk_attn(q, k, v, t.kv_off, w.prefix, w.budget, idx, out=out)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert Bd.device_error() == 0
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            Bd.quoka_select(q, k, t.kv_off, w.prefix, w.nq, w.budget, b_max, idx_out=idx,
+                            workspace=ws)
+            e1.record(stream)
+            Bd.sparse_chunk_attn(q, k, v, t.kv_off, w.prefix, w.budget, idx, out=out)
+            e2.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sel_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    att_ms = [b.elapsed_time(c) for _, b, c in ev]
+    step_ms = [a + b for a, b in zip(sel_ms, att_ms)]
+    total_s = sum(step_ms) / 1e3
+    assert Bd.device_error() == 0
+
+    # end to end through host buffers: the step's new inputs (Q and the chunk's own K/V
+    # rows) go host->device from pinned memory, the output comes back device->host.
+    C = w.chunk
+    q_h = t.q.pin_memory()
+    kv_rows = [(t.kv_off[b] + w.prefix[b], t.kv_off[b] + w.prefix[b] + C) for b in range(w.batch)]
+    kc_h = [t.k_cache[:, a:b_].contiguous().pin_memory() for a, b_ in kv_rows]
+    vc_h = [t.v_cache[:, a:b_].contiguous().pin_memory() for a, b_ in kv_rows]
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = q_h.numel() * q_h.element_size() + sum(2 * x.numel() * x.element_size() for x in kc_h)
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        for (a, b_), kh, vh in zip(kv_rows, kc_h, vc_h):
+            k[:, a:b_].copy_(kh, non_blocking=True)
+            v[:, a:b_].copy_(vh, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        flush.zero_()
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b_.record(stream)
+        b_.synchronize()
+        e2e_ms.append(a.elapsed_time(b_))
+    assert torch.equal(out_h.to(dev), out)
+
+    tokens = w.batch * C
+    if world > 1:
+        m = torch.tensor([total_s, sum(e2e_ms) / 1e3], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(m, op=torch.distributed.ReduceOp.MAX)
+        total_s, e2e_total_s = m.tolist()
+    else:
+        e2e_total_s = sum(e2e_ms) / 1e3
+    value = world * args.steps * tokens / total_s
+    e2e_value = world * args.steps * tokens / e2e_total_s
+
+    st = stage_model(w)
+    rl = roofline_us(st, peaks)
+    att_avg_s = statistics.mean(att_ms) / 1e3
+    achieved = st["attn"]["flops"] / att_avg_s / 1e12
+    path_roof_us = sum(rl.values())
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_s * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "chunk": C, "prefix": list(w.prefix),
+                   "h_q": w.h_q, "h_kv": w.h_kv, "head_dim": w.head_dim, "nq": w.nq,
+                   "budget": list(w.budget), "l2": "256 MB flush before every timed step",
+                   "parallelism": f"independent chunk step per GPU x{world}"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "stage_us": {"select": statistics.mean(sel_ms) * 1e3,
+                     "attn": statistics.mean(att_ms) * 1e3},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": None, "kernel": "sparse_chunk_attn",
+                     "peak_source": f"{peak_src} bf16 dense (burst)"},
+        "path_roofline": {"roofline_us": path_roof_us, "stage_roofline_us": rl,
+                          "measured_us": total_s * 1e6 / args.steps,
+                          "frac": path_roof_us / (total_s * 1e6 / args.steps)},
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = oracle_sample(w, t)
+        line["cpu_baseline"] = {"value": r["tokens_per_s"], "unit": UNIT, "cores": blas_threads(),
+                                "kind": "oracle", "sample": r["sample"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = W.WORKLOADS[args.workload]
+    if w.prompt_chunks != 1:
+        raise SystemExit("bench.py times single-chunk workloads")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,165 @@
+/*
+ * quoka.h - C ABI of libquoka.so: query-oriented KV selection followed by sparse
+ * attention for one chunk of a chunked LLM prefill, on one NVIDIA B200 (sm_100a).
+ *
+ * The problem statement follows the QUOKA page ("Qualcomm QuoKA ...", arXiv
+ * 2602.08722): Figure 1(a) - every chunk of a chunked prefill first sub-selects the
+ * KV cache, and the compacted cache is then fed to a dense attention kernel;
+ * Figure 1(b) and the method summary - selection filters the chunk's queries by
+ * cosine dissimilarity to their mean, scores keys by query-key cosine similarity,
+ * and aggregates with max pooling over queries and mean pooling over the query
+ * heads of a GQA group.  KV-head sharing (MQA / GQA) follows the "Multi-Query
+ * Attention" page, technical insight section.  The QUILT page (shared-query
+ * execution) motivates loading each selected K/V row once per chunk and reusing it
+ * for every query of the group.
+ *
+ * Conventions for every call
+ *   - All memory is owned by the caller.  The library allocates and frees nothing.
+ *   - Device pointers must be 16-byte aligned; `workspace` must be 256-byte aligned.
+ *   - Host arrays (kv_off, prefix_len, budget) are read before the call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Arguments are validated on the host before any launch: a failed
+ *     check returns a non-OK status, launches nothing and leaves outputs untouched.
+ *     quoka_last_error() then describes the failure (thread-local string).
+ *   - Launch failures return QUOKA_ERR_CUDA.  Kernels never trap; a kernel that
+ *     gives up a bounded wait records a nonzero code readable through
+ *     quoka_device_error().
+ *   - Tensor layouts (row-major, innermost dimension last):
+ *       q_chunk  [batch, h_q, chunk, head_dim]               (dtype)
+ *       k_cache  [h_kv, kv_off[batch], head_dim]             (dtype)
+ *       v_cache  [h_kv, kv_off[batch], head_dim]             (dtype)
+ *     Sequence b owns cache rows [kv_off[b], kv_off[b+1]).  Its prefix (the tokens
+ *     of earlier chunks) is rows kv_off[b] .. kv_off[b]+prefix_len[b]-1, and the
+ *     chunk's own K/V (already written by the caller) follow at
+ *     kv_off[b]+prefix_len[b]+t for chunk position t.
+ *   - Query head h uses KV head h / (h_q / h_kv).
+ */
+#ifndef QUOKA_H
+#define QUOKA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QUOKA_OK = 0,
+  QUOKA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or offset     */
+  QUOKA_ERR_UNSUPPORTED = 2,   /* valid but unsupported: head_dim, batch, chunk    */
+  QUOKA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required        */
+  QUOKA_ERR_CUDA = 4           /* a CUDA runtime call or launch failed              */
+} quoka_status;
+
+typedef enum { QUOKA_F32 = 0, QUOKA_BF16 = 1 } quoka_dtype;
+
+#define QUOKA_MAX_BATCH 64     /* sequences per call                                 */
+#define QUOKA_MAX_CHUNK 8192   /* chunk tokens per sequence                          */
+#define QUOKA_MAX_GROUP 64     /* query heads per KV head                            */
+
+typedef struct {
+  int batch;          /* sequences in this chunk step, 1..QUOKA_MAX_BATCH           */
+  int h_q;            /* query heads                                                */
+  int h_kv;           /* KV heads; h_q % h_kv == 0, h_q / h_kv <= QUOKA_MAX_GROUP   */
+  int head_dim;       /* 64 or 128                                                  */
+  int chunk;          /* C, chunk tokens per sequence, 1..QUOKA_MAX_CHUNK           */
+  quoka_dtype dtype;  /* element type of q_chunk, k_cache, v_cache and out          */
+} quoka_shape;
+
+/*
+ * Bytes of device scratch quoka_select() needs for prefixes up to `max_prefix` and
+ * `nq` kept queries per head.  Returns 0 for an invalid shape.  The scratch holds
+ * the gathered kept queries with their inverse norms and one fp32 pooled score per
+ * prefix key and KV head (the full query-key score matrix is never stored).
+ */
+size_t quoka_select_workspace_size(const quoka_shape* shape, int max_prefix, int nq);
+
+/*
+ * Byte offset and row stride (in floats) of the pooled key scores inside the
+ * workspace of quoka_select(): after a call, scores of sequence b, KV head g, key j
+ * are at ((float*)(ws + offset))[(b * h_kv + g) * row_stride + j].  For tests and
+ * diagnostics only.
+ */
+quoka_status quoka_workspace_pooled_view(const quoka_shape* shape, int max_prefix, int nq,
+                                         size_t* offset, size_t* row_stride);
+
+/*
+ * quoka_select - QUOKA KV selection for one chunk step (QUOKA page: Figure 1(b) and
+ * the method summary's three steps; Figure 2 for the direction of the query filter).
+ *
+ * Per sequence b and query head h, with C = shape->chunk, P = prefix_len[b]:
+ *   1. m_h = mean over t < C of q_t / |q_t|                        (mean query)
+ *   2. keep the Nk = min(nq, C) queries with the smallest cos(q_t, m_h), ties to the
+ *      lower t                                                   (query subselection)
+ * Per KV head g with heads H_g = {g*G .. g*G+G-1}, for every prefix key j < P:
+ *   3. s_j = (1/G) * sum_{h in H_g} max_{i kept in h} cos(q_i, k_j)
+ *                                  (cosine scoring; max then mean group pooling)
+ *   4. keep the min(budget[b], P) keys with the largest s_j, ties to the lower j.
+ * A zero-norm query or key has cosine 0.  The chunk's own keys are never candidates:
+ * the attention call always adds them causally, so budget[b] counts prefix keys.
+ *
+ *   q_chunk     device, [batch, h_q, chunk, head_dim]
+ *   k_cache     device, [h_kv, kv_off[batch], head_dim]
+ *   kv_off      host, batch + 1 nondecreasing row offsets, kv_off[0] >= 0,
+ *               kv_off[b+1] - kv_off[b] >= prefix_len[b] + chunk
+ *   prefix_len  host, batch entries, 0 <= P
+ *   nq          kept queries per query head, >= 1 (values above chunk keep all)
+ *   budget      host, batch entries, 0 <= budget[b] <= b_max
+ *   b_max       row length of idx_out, >= 1
+ *   idx_out     device int32 [batch, h_kv, b_max]: the kept prefix positions
+ *               (relative to the sequence's first row) in ascending order, then -1
+ *   kept_out    device int32 [batch, h_q, nq] or NULL: kept chunk positions in
+ *               ascending order, then -1 when nq > chunk
+ *   workspace   device scratch of quoka_select_workspace_size(shape, max_b P, nq)
+ *               bytes; contents on entry are ignored
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE (ws_bytes too small), CUDA.
+ */
+quoka_status quoka_select(const quoka_shape* shape, const void* q_chunk, const void* k_cache,
+                          const int64_t* kv_off, const int32_t* prefix_len, int nq,
+                          const int32_t* budget, int b_max, int32_t* idx_out,
+                          int32_t* kept_out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * sparse_chunk_attn - dense attention of the chunk over the compacted cache
+ * (QUOKA page, Figure 1(a): the compacted KV cache is fed to a dense attention
+ * kernel; QUILT page: each shared K/V row is loaded once and reused by every query
+ * that selected it - here the G query heads of a KV head share one selection).
+ *
+ * Query t of head h (KV head g = h / G) of sequence b attends to
+ *     keys  { idx[b, g, i] : i < n_b }  U  { P + u : 0 <= u <= t }
+ * with n_b = min(budget[b], P) and P = prefix_len[b], computing
+ *     out = softmax(q . k^T / sqrt(head_dim)) . v
+ * with fp32 accumulation and fp32 softmax, stored in `dtype`.
+ *
+ *   q_chunk, k_cache, v_cache, kv_off, prefix_len   as for quoka_select
+ *   budget      host, batch entries, 0 <= budget[b] <= b_max (as for quoka_select)
+ *   idx         device int32 [batch, h_kv, b_max], e.g. quoka_select's idx_out;
+ *               entries [0, n_b) must be distinct prefix positions in [0, P)
+ *   out         device [batch, h_q, chunk, head_dim]; must not alias an input
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.  idx entries are not range-checked on the
+ * device; an entry outside [0, P) is a caller error.
+ */
+quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk,
+                               const void* k_cache, const void* v_cache,
+                               const int64_t* kv_off, const int32_t* prefix_len,
+                               const int32_t* budget, const int32_t* idx, int b_max,
+                               void* out, void* stream);
+
+/* Thread-local description of the last non-OK status returned on this thread. */
+const char* quoka_last_error(void);
+
+/*
+ * Reads and clears the device error word (0 = no kernel gave up a bounded wait).
+ * Synchronises `stream`.  Returns QUOKA_ERR_CUDA if the read itself fails.
+ */
+quoka_status quoka_device_error(uint32_t* code, void* stream);
+
+/* Library ABI version (major * 100 + minor). */
+int quoka_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QUOKA_H */

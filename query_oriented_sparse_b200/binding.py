@@ -1,0 +1,174 @@
+"""ctypes binding over libquoka.so (argument marshalling only).
+
+Every step of the selection and attention runs in the library's CUDA kernels; this
+module turns torch tensors into pointers, host arrays and the current torch stream,
+and turns non-OK statuses into exceptions.  torch provides device memory and streams.
+If the library is missing the first call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libquoka.so")
+
+QUOKA_OK, QUOKA_ERR_INVALID_ARG, QUOKA_ERR_UNSUPPORTED, QUOKA_ERR_WORKSPACE, QUOKA_ERR_CUDA = range(5)
+QUOKA_F32, QUOKA_BF16 = 0, 1
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA"}
+
+# (name, restype, argtypes) of every symbol include/quoka.h declares
+_P = ctypes.c_void_p
+_I64P = ctypes.POINTER(ctypes.c_int64)
+_I32P = ctypes.POINTER(ctypes.c_int32)
+
+
+class QuokaShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("h_q", ctypes.c_int), ("h_kv", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("chunk", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+_SHAPE_P = ctypes.POINTER(QuokaShape)
+
+SIGNATURES = {
+    "quoka_version": (ctypes.c_int, []),
+    "quoka_last_error": (ctypes.c_char_p, []),
+    "quoka_select_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int, ctypes.c_int]),
+    "quoka_workspace_pooled_view": (ctypes.c_int, [_SHAPE_P, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.POINTER(ctypes.c_size_t),
+                                                   ctypes.POINTER(ctypes.c_size_t)]),
+    "quoka_select": (ctypes.c_int, [_SHAPE_P, _P, _P, _I64P, _I32P, ctypes.c_int, _I32P,
+                                    ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
+    "sparse_chunk_attn": (ctypes.c_int, [_SHAPE_P, _P, _P, _P, _I64P, _I32P, _I32P, _P,
+                                         ctypes.c_int, _P, _P]),
+    "quoka_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
+}
+
+_lib = None
+
+
+class QuokaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libquoka.so from the package directory (raises if it was never built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m query_oriented_sparse_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != QUOKA_OK:
+        raise QuokaError(status, lib().quoka_last_error().decode())
+
+
+def make_shape(batch: int, h_q: int, h_kv: int, head_dim: int, chunk: int,
+               dtype: torch.dtype) -> QuokaShape:
+    if dtype == torch.float32:
+        dt = QUOKA_F32
+    elif dtype == torch.bfloat16:
+        dt = QUOKA_BF16
+    else:
+        raise QuokaError(QUOKA_ERR_UNSUPPORTED, f"dtype {dtype}")
+    return QuokaShape(batch, h_q, h_kv, head_dim, chunk, dt)
+
+
+def shape_of(q_chunk: torch.Tensor, k_cache: torch.Tensor) -> QuokaShape:
+    batch, h_q, chunk, d = q_chunk.shape
+    return make_shape(batch, h_q, k_cache.shape[0], d, chunk, q_chunk.dtype)
+
+
+def _host_i64(xs: Sequence[int]):
+    arr = (ctypes.c_int64 * len(xs))(*[int(x) for x in xs])
+    return arr
+
+
+def _host_i32(xs: Sequence[int]):
+    return (ctypes.c_int32 * len(xs))(*[int(x) for x in xs])
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def version() -> int:
+    return lib().quoka_version()
+
+
+def select_workspace_size(shape: QuokaShape, max_prefix: int, nq: int) -> int:
+    return int(lib().quoka_select_workspace_size(ctypes.byref(shape), max_prefix, nq))
+
+
+def pooled_view(workspace: torch.Tensor, shape: QuokaShape, max_prefix: int, nq: int) -> torch.Tensor:
+    """The pooled key scores inside a quoka_select workspace, [batch, h_kv, stride] fp32."""
+    off, stride = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().quoka_workspace_pooled_view(ctypes.byref(shape), max_prefix, nq,
+                                             ctypes.byref(off), ctypes.byref(stride)))
+    n = shape.batch * shape.h_kv * stride.value
+    return workspace[off.value:off.value + 4 * n].view(torch.float32).view(
+        shape.batch, shape.h_kv, stride.value)
+
+
+def quoka_select(q_chunk: torch.Tensor, k_cache: torch.Tensor, kv_off: Sequence[int],
+                 prefix_len: Sequence[int], nq: int, budget: Sequence[int],
+                 b_max: Optional[int] = None, idx_out: Optional[torch.Tensor] = None,
+                 kept_out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """QUOKA selection for one chunk step; returns idx [batch, h_kv, b_max] int32."""
+    shape = shape_of(q_chunk, k_cache)
+    if b_max is None:
+        b_max = max(max(int(b) for b in budget), 1)
+    dev = q_chunk.device
+    if idx_out is None:
+        idx_out = torch.empty(shape.batch, shape.h_kv, b_max, dtype=torch.int32, device=dev)
+    if workspace is None:
+        ws = select_workspace_size(shape, max(int(p) for p in prefix_len), nq)
+        workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+    _check(lib().quoka_select(
+        ctypes.byref(shape), _ptr(q_chunk), _ptr(k_cache), _host_i64(kv_off),
+        _host_i32(prefix_len), int(nq), _host_i32(budget), int(b_max), _ptr(idx_out),
+        _ptr(kept_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        ctypes.c_void_p(_stream(stream))))
+    return idx_out
+
+
+def sparse_chunk_attn(q_chunk: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      kv_off: Sequence[int], prefix_len: Sequence[int], budget: Sequence[int],
+                      idx: torch.Tensor, out: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Attention of the chunk over its compacted cache; returns out [batch, h_q, C, d]."""
+    shape = shape_of(q_chunk, k_cache)
+    if out is None:
+        out = torch.empty_like(q_chunk)
+    _check(lib().sparse_chunk_attn(
+        ctypes.byref(shape), _ptr(q_chunk), _ptr(k_cache), _ptr(v_cache), _host_i64(kv_off),
+        _host_i32(prefix_len), _host_i32(budget), _ptr(idx), int(idx.shape[-1]), _ptr(out),
+        ctypes.c_void_p(_stream(stream))))
+    return out
+
+
+def device_error(stream: Optional[torch.cuda.Stream] = None) -> int:
+    code = ctypes.c_uint32(0)
+    _check(lib().quoka_device_error(ctypes.byref(code), ctypes.c_void_p(_stream(stream))))
+    return code.value

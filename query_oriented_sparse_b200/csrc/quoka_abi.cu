@@ -1,0 +1,277 @@
+// Host side of libquoka.so: argument validation, workspace layout and kernel launches
+// behind the C ABI declared in include/quoka.h.  Every check runs before any CUDA
+// call, so an invalid call launches nothing.
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "common.cuh"
+#include "qsub.cuh"
+#include "score_simt.cuh"
+#include "topk.cuh"
+#include "attn_simt.cuh"
+
+using namespace quoka;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+quoka_status fail(quoka_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+quoka_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(QUOKA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+struct Dims {
+  int batch, h_q, h_kv, G, D, C;
+  quoka_dtype dt;
+  int esz;
+};
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+quoka_status check_shape(const quoka_shape* s, Dims* d) {
+  if (!s) return fail(QUOKA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 1) return fail(QUOKA_ERR_INVALID_ARG, "batch must be >= 1 (got %d)", s->batch);
+  if (s->batch > QUOKA_MAX_BATCH)
+    return fail(QUOKA_ERR_UNSUPPORTED, "batch %d exceeds QUOKA_MAX_BATCH=%d", s->batch, QUOKA_MAX_BATCH);
+  if (s->h_q < 1 || s->h_kv < 1 || s->h_q % s->h_kv != 0)
+    return fail(QUOKA_ERR_INVALID_ARG, "h_q=%d must be a positive multiple of h_kv=%d", s->h_q, s->h_kv);
+  if (s->h_q / s->h_kv > QUOKA_MAX_GROUP)
+    return fail(QUOKA_ERR_UNSUPPORTED, "group size %d exceeds %d", s->h_q / s->h_kv, QUOKA_MAX_GROUP);
+  if (s->head_dim != 64 && s->head_dim != 128)
+    return fail(QUOKA_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", s->head_dim);
+  if (s->chunk < 1) return fail(QUOKA_ERR_INVALID_ARG, "chunk must be >= 1 (got %d)", s->chunk);
+  if (s->chunk > QUOKA_MAX_CHUNK)
+    return fail(QUOKA_ERR_UNSUPPORTED, "chunk %d exceeds QUOKA_MAX_CHUNK=%d", s->chunk, QUOKA_MAX_CHUNK);
+  if (s->dtype != QUOKA_F32 && s->dtype != QUOKA_BF16)
+    return fail(QUOKA_ERR_UNSUPPORTED, "unknown dtype %d", (int)s->dtype);
+  d->batch = s->batch;
+  d->h_q = s->h_q;
+  d->h_kv = s->h_kv;
+  d->G = s->h_q / s->h_kv;
+  d->D = s->head_dim;
+  d->C = s->chunk;
+  d->dt = s->dtype;
+  d->esz = s->dtype == QUOKA_F32 ? 4 : 2;
+  return QUOKA_OK;
+}
+
+// Fills the kernel-side sequence table from the host arrays.
+quoka_status build_table(const Dims& d, const int64_t* kv_off, const int32_t* prefix,
+                         const int32_t* budget, int b_max, SeqTable* tab, long long* rows) {
+  if (!kv_off || !prefix || !budget) return fail(QUOKA_ERR_INVALID_ARG, "kv_off, prefix_len and budget must be non-NULL");
+  if (b_max < 1) return fail(QUOKA_ERR_INVALID_ARG, "b_max must be >= 1 (got %d)", b_max);
+  if (kv_off[0] < 0) return fail(QUOKA_ERR_INVALID_ARG, "kv_off[0] must be >= 0");
+  tab->batch = d.batch;
+  tab->max_prefix = 0;
+  for (int b = 0; b <= d.batch; ++b) tab->kv_off[b] = kv_off[b];
+  for (int b = 0; b < d.batch; ++b) {
+    const int P = prefix[b];
+    if (P < 0) return fail(QUOKA_ERR_INVALID_ARG, "prefix_len[%d] = %d < 0", b, P);
+    if (budget[b] < 0 || budget[b] > b_max)
+      return fail(QUOKA_ERR_INVALID_ARG, "budget[%d] = %d outside [0, b_max=%d]", b, budget[b], b_max);
+    if (kv_off[b + 1] - kv_off[b] < (int64_t)P + d.C)
+      return fail(QUOKA_ERR_INVALID_ARG,
+                  "sequence %d owns %lld cache rows, fewer than prefix_len + chunk = %lld", b,
+                  (long long)(kv_off[b + 1] - kv_off[b]), (long long)P + d.C);
+    tab->prefix[b] = P;
+    tab->nsel[b] = budget[b] < P ? budget[b] : P;
+    if (P > tab->max_prefix) tab->max_prefix = P;
+  }
+  for (int b = d.batch; b < QUOKA_MAX_BATCH; ++b) { tab->prefix[b] = 0; tab->nsel[b] = 0; }
+  *rows = kv_off[d.batch];
+  return QUOKA_OK;
+}
+
+struct WsLayout {
+  size_t qsel, qinv, pooled, total;
+  long long pooled_stride;  // floats per (sequence, KV head) row
+  int nk;
+};
+
+WsLayout ws_layout(const Dims& d, int max_prefix, int nq) {
+  WsLayout w;
+  w.nk = nq < d.C ? nq : d.C;
+  size_t off = 0;
+  w.qsel = off;
+  off = align_up(off + (size_t)d.batch * d.h_q * w.nk * d.D * d.esz, 256);
+  w.qinv = off;
+  off = align_up(off + (size_t)d.batch * d.h_q * w.nk * 4, 256);
+  w.pooled_stride = (long long)align_up((size_t)(max_prefix > 0 ? max_prefix : 1), 128);
+  w.pooled = off;
+  off = align_up(off + (size_t)d.batch * d.h_kv * w.pooled_stride * 4, 256);
+  w.total = off;
+  return w;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+cudaError_t ensure_smem(K kernel, int bytes) {
+  static int done_for[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && done_for[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev < 64) done_for[dev] = bytes;
+  return e;
+}
+
+template <typename T, int D>
+quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                           const void* k, int nq, int b_max, int32_t* idx_out, int32_t* kept_out,
+                           unsigned char* ws, const WsLayout& w, cudaStream_t st) {
+  T* qsel = reinterpret_cast<T*>(ws + w.qsel);
+  float* qinv = reinterpret_cast<float*>(ws + w.qinv);
+  float* pooled = reinterpret_cast<float*>(ws + w.pooled);
+  cudaError_t e;
+
+  const int s1 = qsub_smem_bytes<D>(d.C);
+  if ((e = ensure_smem(qsub_kernel<T, D>, s1)) != cudaSuccess) return cuda_fail(e, "qsub smem");
+  qsub_kernel<T, D><<<d.batch * d.h_q, QSUB_THREADS, s1, st>>>(
+      reinterpret_cast<const T*>(q), d.h_q, d.C, w.nk, nq, kept_out, qsel, qinv);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "qsub launch");
+
+  if (tab.max_prefix > 0) {
+    const int s2 = score_simt_smem_bytes<D>(d.G);
+    if ((e = ensure_smem(score_simt_kernel<T, D>, s2)) != cudaSuccess) return cuda_fail(e, "score smem");
+    dim3 grid((tab.max_prefix + SCS_KEYS - 1) / SCS_KEYS, d.h_kv, d.batch);
+    score_simt_kernel<T, D><<<grid, SCS_THREADS, s2, st>>>(
+        reinterpret_cast<const T*>(k), rows, tab, d.h_kv, d.G, w.nk, qsel, qinv, pooled,
+        w.pooled_stride);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score launch");
+  }
+
+  topk_kernel<<<d.batch * d.h_kv * TOPK_CS, TOPK_THREADS, 0, st>>>(pooled, w.pooled_stride, tab,
+                                                                   d.h_kv, b_max, idx_out);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
+  return QUOKA_OK;
+}
+
+template <typename T, int D>
+quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                         const void* k, const void* v, const int32_t* idx, int b_max, void* out,
+                         cudaStream_t st) {
+  cudaError_t e;
+  const int s = attn_simt_smem_bytes<D>();
+  if ((e = ensure_smem(attn_simt_kernel<T, D>, s)) != cudaSuccess) return cuda_fail(e, "attn smem");
+  dim3 grid((d.C + ATS_ROWS - 1) / ATS_ROWS, d.h_q, d.batch);
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  attn_simt_kernel<T, D><<<grid, ATS_THREADS, s, st>>>(
+      reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(k), reinterpret_cast<const T*>(v),
+      rows, tab, d.h_q, d.h_kv, d.C, idx, b_max, reinterpret_cast<T*>(out), scale_log2);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn launch");
+  return QUOKA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int quoka_version(void) { return 100; }
+
+const char* quoka_last_error(void) { return g_last_error.c_str(); }
+
+size_t quoka_select_workspace_size(const quoka_shape* shape, int max_prefix, int nq) {
+  Dims d;
+  if (check_shape(shape, &d) != QUOKA_OK || max_prefix < 0 || nq < 1) return 0;
+  return ws_layout(d, max_prefix, nq).total;
+}
+
+quoka_status quoka_workspace_pooled_view(const quoka_shape* shape, int max_prefix, int nq,
+                                         size_t* offset, size_t* row_stride) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (max_prefix < 0 || nq < 1 || !offset || !row_stride)
+    return fail(QUOKA_ERR_INVALID_ARG, "bad max_prefix/nq or NULL output");
+  const WsLayout w = ws_layout(d, max_prefix, nq);
+  *offset = w.pooled;
+  *row_stride = (size_t)w.pooled_stride;
+  return QUOKA_OK;
+}
+
+quoka_status quoka_select(const quoka_shape* shape, const void* q_chunk, const void* k_cache,
+                          const int64_t* kv_off, const int32_t* prefix_len, int nq,
+                          const int32_t* budget, int b_max, int32_t* idx_out, int32_t* kept_out,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (!q_chunk || !k_cache || !idx_out) return fail(QUOKA_ERR_INVALID_ARG, "q_chunk, k_cache and idx_out must be non-NULL");
+  if (!aligned(q_chunk, 16) || !aligned(k_cache, 16) || !aligned(idx_out, 16) ||
+      (kept_out && !aligned(kept_out, 16)))
+    return fail(QUOKA_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (nq < 1) return fail(QUOKA_ERR_INVALID_ARG, "nq must be >= 1 (got %d)", nq);
+  SeqTable tab;
+  long long rows = 0;
+  if ((s = build_table(d, kv_off, prefix_len, budget, b_max, &tab, &rows)) != QUOKA_OK) return s;
+  const WsLayout w = ws_layout(d, tab.max_prefix, nq);
+  if (!workspace) return fail(QUOKA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", w.total);
+  if (!aligned(workspace, 256)) return fail(QUOKA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < w.total)
+    return fail(QUOKA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, w.total);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+  if (d.dt == QUOKA_F32) {
+    return d.D == 64 ? launch_select<float, 64>(d, tab, rows, q_chunk, k_cache, nq, b_max, idx_out, kept_out, ws, w, st)
+                     : launch_select<float, 128>(d, tab, rows, q_chunk, k_cache, nq, b_max, idx_out, kept_out, ws, w, st);
+  }
+  return d.D == 64 ? launch_select<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_cache, nq, b_max, idx_out, kept_out, ws, w, st)
+                   : launch_select<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, nq, b_max, idx_out, kept_out, ws, w, st);
+}
+
+quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk, const void* k_cache,
+                               const void* v_cache, const int64_t* kv_off,
+                               const int32_t* prefix_len, const int32_t* budget,
+                               const int32_t* idx, int b_max, void* out, void* stream) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (!q_chunk || !k_cache || !v_cache || !idx || !out)
+    return fail(QUOKA_ERR_INVALID_ARG, "q_chunk, k_cache, v_cache, idx and out must be non-NULL");
+  if (!aligned(q_chunk, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(idx, 16) ||
+      !aligned(out, 16))
+    return fail(QUOKA_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (out == q_chunk || out == k_cache || out == v_cache)
+    return fail(QUOKA_ERR_INVALID_ARG, "out must not alias an input");
+  SeqTable tab;
+  long long rows = 0;
+  if ((s = build_table(d, kv_off, prefix_len, budget, b_max, &tab, &rows)) != QUOKA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.dt == QUOKA_F32) {
+    return d.D == 64 ? launch_attn<float, 64>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, st)
+                     : launch_attn<float, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, st);
+  }
+  return d.D == 64 ? launch_attn<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, st)
+                   : launch_attn<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, st);
+}
+
+quoka_status quoka_device_error(uint32_t* code, void* stream) {
+  if (!code) return fail(QUOKA_ERR_INVALID_ARG, "code is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof(v), 0, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  *code = v;
+  return QUOKA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+"""The C ABI library: it loads, exports every symbol include/quoka.h declares, and its
+host-side validation rejects bad calls with the documented status before launching
+anything.  The fake-pointer cases run only where no GPU is present (on a GPU machine the
+same rejections are exercised with real buffers in test_kernels.py)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from query_oriented_sparse_b200 import binding as Bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "quoka.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", src)) -
+                  {"if", "sizeof", "defined"})
+
+
+def test_header_declares_the_boundary():
+    fns = declared_functions()
+    for name in ("quoka_select", "sparse_chunk_attn", "quoka_select_workspace_size",
+                 "quoka_last_error", "quoka_device_error", "quoka_version",
+                 "quoka_workspace_pooled_view"):
+        assert name in fns
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = Bd.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libquoka.so does not export {name}"
+    assert set(declared_functions()) == set(Bd.SIGNATURES), "binding and header disagree"
+    assert Bd.version() == 100
+
+
+def test_workspace_size_is_host_only():
+    s = Bd.make_shape(1, 32, 8, 128, 4096, torch.bfloat16)
+    n = Bd.select_workspace_size(s, 131072, 128)
+    # kept queries (32*128 rows of 256 B) + their inverse norms + 8*131072 fp32 scores
+    assert n >= 32 * 128 * 256 + 32 * 128 * 4 + 8 * 131072 * 4
+    assert n % 256 == 0
+    bad = Bd.make_shape(1, 32, 8, 96, 4096, torch.bfloat16)
+    assert Bd.select_workspace_size(bad, 10, 4) == 0
+
+
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(),
+                            reason="fake device pointers are only passed where there is no GPU")
+
+FAKE = 0x10000  # never dereferenced: every case below must fail host-side validation
+
+
+def _select(shape, q=FAKE, k=FAKE, kv_off=(0, 1024), prefix=(512,), nq=8, budget=(64,),
+            b_max=64, idx=FAKE, kept=None, ws=FAKE, ws_bytes=1 << 30):
+    lib = Bd.lib()
+    return lib.quoka_select(ctypes.byref(shape), q, k, Bd._host_i64(kv_off), Bd._host_i32(prefix),
+                            nq, Bd._host_i32(budget), b_max, idx, kept, ws, ws_bytes, None)
+
+
+def _attn(shape, q=FAKE, k=FAKE, v=FAKE, kv_off=(0, 1024), prefix=(512,), budget=(64,),
+          idx=FAKE, b_max=64, out=FAKE + 4096):
+    lib = Bd.lib()
+    return lib.sparse_chunk_attn(ctypes.byref(shape), q, k, v, Bd._host_i64(kv_off),
+                                 Bd._host_i32(prefix), Bd._host_i32(budget), idx, b_max, out, None)
+
+
+@no_gpu
+@pytest.mark.parametrize("case,status", [
+    (dict(shape=dict(head_dim=96)), Bd.QUOKA_ERR_UNSUPPORTED),
+    (dict(shape=dict(batch=65)), Bd.QUOKA_ERR_UNSUPPORTED),
+    (dict(shape=dict(batch=0)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(shape=dict(h_q=6, h_kv=4)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(shape=dict(chunk=9000)), Bd.QUOKA_ERR_UNSUPPORTED),
+    (dict(shape=dict(dtype=7)), Bd.QUOKA_ERR_UNSUPPORTED),
+    (dict(q=FAKE + 2), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(idx=None), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(nq=0), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(prefix=(-1,)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(prefix=(1000,)), Bd.QUOKA_ERR_INVALID_ARG),        # prefix + chunk > rows
+    (dict(budget=(65,)), Bd.QUOKA_ERR_INVALID_ARG),          # budget > b_max
+    (dict(b_max=0, budget=(0,)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(ws=None), Bd.QUOKA_ERR_WORKSPACE),
+    (dict(ws_bytes=100), Bd.QUOKA_ERR_WORKSPACE),
+    (dict(ws=FAKE + 16), Bd.QUOKA_ERR_INVALID_ARG),          # workspace not 256-aligned
+    (dict(kv_off=(-4, 1020)), Bd.QUOKA_ERR_INVALID_ARG),
+])
+def test_select_rejects(case, status):
+    shp = dict(batch=1, h_q=8, h_kv=2, head_dim=128, chunk=256, dtype=Bd.QUOKA_BF16)
+    shp.update(case.pop("shape", {}))
+    shape = Bd.QuokaShape(**shp)
+    assert _select(shape, **case) == status
+    assert Bd.lib().quoka_last_error().decode()
+
+
+@no_gpu
+@pytest.mark.parametrize("case,status", [
+    (dict(shape=dict(head_dim=32)), Bd.QUOKA_ERR_UNSUPPORTED),
+    (dict(out=FAKE), Bd.QUOKA_ERR_INVALID_ARG),               # aliases q
+    (dict(v=None), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(k=FAKE + 8), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(budget=(-1,)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(kv_off=(0, 600)), Bd.QUOKA_ERR_INVALID_ARG),
+])
+def test_attn_rejects(case, status):
+    shp = dict(batch=1, h_q=8, h_kv=2, head_dim=128, chunk=256, dtype=Bd.QUOKA_BF16)
+    shp.update(case.pop("shape", {}))
+    shape = Bd.QuokaShape(**shp)
+    assert _attn(shape, **case) == status
+
+
+def test_null_shape_rejected():
+    lib = Bd.lib()
+    assert lib.quoka_select(None, FAKE, FAKE, Bd._host_i64((0, 8)), Bd._host_i32((0,)), 1,
+                            Bd._host_i32((0,)), 1, FAKE, None, FAKE, 1 << 20, None) == \
+        Bd.QUOKA_ERR_INVALID_ARG
+    assert "NULL" in lib.quoka_last_error().decode()
