@@ -3,7 +3,10 @@
 // call, so an invalid call launches nothing.
 #include <cstdarg>
 #include <cstdio>
+#include <map>
+#include <mutex>
 #include <string>
+#include <utility>
 
 #include "common.cuh"
 #include "qsub.cuh"
@@ -116,16 +119,21 @@ WsLayout ws_layout(const Dims& d, int max_prefix, int nq) {
   return w;
 }
 
-// Raises a kernel's dynamic shared-memory limit once per device.
+// Raises a kernel's dynamic shared-memory limit, once per (kernel, device).
+std::mutex g_smem_mu;
+std::map<std::pair<const void*, int>, int> g_smem_set;
+
 template <typename K>
 cudaError_t ensure_smem(K kernel, int bytes) {
-  static int done_for[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 64 && done_for[dev] >= bytes) return cudaSuccess;
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lock(g_smem_mu);
+  auto it = g_smem_set.find(key);
+  if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev < 64) done_for[dev] = bytes;
+  if (e == cudaSuccess) g_smem_set[key] = bytes;
   return e;
 }
 
