@@ -146,6 +146,32 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk,
                                const int32_t* budget, const int32_t* idx, int b_max,
                                void* out, void* stream);
 
+/*
+ * quoka_select_noalloc - quoka_select without a caller-provided workspace.
+ *
+ * The paper has no counterpart to this call; it exists for callers that cannot
+ * allocate device memory at the point where they run the selection: for example a
+ * plugin inside a serving engine that reserved nearly all HBM for its KV cache at
+ * start-up and hands plugins no allocator, or a latency-critical path where the
+ * device synchronisation implied by cudaMalloc/cudaFree is not acceptable.
+ *
+ * Same arguments, semantics and errors as quoka_select, minus workspace/ws_bytes.
+ * The scratch lives in one fixed device array of QUOKA_NOALLOC_SCRATCH_BYTES inside
+ * the library, reserved on every GPU that loads the library until the process
+ * exits.  A call whose quoka_select_workspace_size() would exceed that size returns
+ * QUOKA_ERR_WORKSPACE and launches nothing.  The first call on a device looks up the
+ * array's device address (once per device, with that device current); make that
+ * first call before any stream capture.  All calls share the one array and the
+ * kernels overwrite every scratch byte they read, so nothing needs clearing between
+ * calls - but two calls whose kernels overlap on the GPU (different streams without
+ * ordering between them) race on the array.  The library allocates nothing here.
+ */
+#define QUOKA_NOALLOC_SCRATCH_BYTES (32u << 20)
+quoka_status quoka_select_noalloc(const quoka_shape* shape, const void* q_chunk,
+                                  const void* k_cache, const int64_t* kv_off,
+                                  const int32_t* prefix_len, int nq, const int32_t* budget,
+                                  int b_max, int32_t* idx_out, int32_t* kept_out, void* stream);
+
 /* Thread-local description of the last non-OK status returned on this thread. */
 const char* quoka_last_error(void);
 

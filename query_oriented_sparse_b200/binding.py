@@ -45,6 +45,8 @@ SIGNATURES = {
     "sparse_chunk_attn": (ctypes.c_int, [_SHAPE_P, _P, _P, _P, _I64P, _I32P, _I32P, _P,
                                          ctypes.c_int, _P, _P]),
     "quoka_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
+    "quoka_select_noalloc": (ctypes.c_int, [_SHAPE_P, _P, _P, _I64P, _I32P, ctypes.c_int, _I32P,
+                                            ctypes.c_int, _P, _P, _P]),
 }
 
 _lib = None
@@ -150,6 +152,26 @@ def quoka_select(q_chunk: torch.Tensor, k_cache: torch.Tensor, kv_off: Sequence[
         _host_i32(prefix_len), int(nq), _host_i32(budget), int(b_max), _ptr(idx_out),
         _ptr(kept_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
         ctypes.c_void_p(_stream(stream))))
+    return idx_out
+
+
+def quoka_select_noalloc(q_chunk: torch.Tensor, k_cache: torch.Tensor, kv_off: Sequence[int],
+                         prefix_len: Sequence[int], nq: int, budget: Sequence[int],
+                         b_max: Optional[int] = None, idx_out: Optional[torch.Tensor] = None,
+                         kept_out: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """quoka_select using the library's built-in scratch instead of a workspace (for
+    callers that cannot allocate device memory); the outputs are still the caller's."""
+    shape = shape_of(q_chunk, k_cache)
+    if b_max is None:
+        b_max = max(max(int(b) for b in budget), 1)
+    if idx_out is None:
+        idx_out = torch.empty(shape.batch, shape.h_kv, b_max, dtype=torch.int32,
+                              device=q_chunk.device)
+    _check(lib().quoka_select_noalloc(
+        ctypes.byref(shape), _ptr(q_chunk), _ptr(k_cache), _host_i64(kv_off),
+        _host_i32(prefix_len), int(nq), _host_i32(budget), int(b_max), _ptr(idx_out),
+        _ptr(kept_out), ctypes.c_void_p(_stream(stream))))
     return idx_out
 
 

@@ -267,6 +267,70 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk, co
                    : launch_attn<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, st);
 }
 
+}  // extern "C"
+
+// ---- allocation-free variant of quoka_select --------------------------------------
+// The scratch is one file-scope device array.  In host code its name is only a
+// host-side stand-in, so its device address is looked up per device with
+// cudaGetSymbolAddress (with that device current) and passed to the kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QUOKA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+std::map<int, void*> g_noalloc_addr;  // device ordinal -> device address of the array
+
+quoka_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  auto it = g_noalloc_addr.find(dev);
+  if (it == g_noalloc_addr.end()) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
+    it = g_noalloc_addr.emplace(dev, p).first;
+  }
+  *out = it->second;
+  return QUOKA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+quoka_status quoka_select_noalloc(const quoka_shape* shape, const void* q_chunk,
+                                  const void* k_cache, const int64_t* kv_off,
+                                  const int32_t* prefix_len, int nq, const int32_t* budget,
+                                  int b_max, int32_t* idx_out, int32_t* kept_out, void* stream) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (!q_chunk || !k_cache || !idx_out) return fail(QUOKA_ERR_INVALID_ARG, "q_chunk, k_cache and idx_out must be non-NULL");
+  if (!aligned(q_chunk, 16) || !aligned(k_cache, 16) || !aligned(idx_out, 16) ||
+      (kept_out && !aligned(kept_out, 16)))
+    return fail(QUOKA_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (nq < 1) return fail(QUOKA_ERR_INVALID_ARG, "nq must be >= 1 (got %d)", nq);
+  SeqTable tab;
+  long long rows = 0;
+  if ((s = build_table(d, kv_off, prefix_len, budget, b_max, &tab, &rows)) != QUOKA_OK) return s;
+  const WsLayout w = ws_layout(d, tab.max_prefix, nq);
+  if (w.total > (size_t)QUOKA_NOALLOC_SCRATCH_BYTES)
+    return fail(QUOKA_ERR_WORKSPACE,
+                "this call needs %zu bytes of scratch; the built-in scratch holds %zu "
+                "(use quoka_select with a caller workspace)", w.total,
+                (size_t)QUOKA_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != QUOKA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = reinterpret_cast<unsigned char*>(scratch);
+  if (d.dt == QUOKA_F32) {
+    return d.D == 64 ? launch_select<float, 64>(d, tab, rows, q_chunk, k_cache, nq, b_max, idx_out, kept_out, ws, w, st)
+                     : launch_select<float, 128>(d, tab, rows, q_chunk, k_cache, nq, b_max, idx_out, kept_out, ws, w, st);
+  }
+  return d.D == 64 ? launch_select<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_cache, nq, b_max, idx_out, kept_out, ws, w, st)
+                   : launch_select<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, nq, b_max, idx_out, kept_out, ws, w, st);
+}
+
 quoka_status quoka_device_error(uint32_t* code, void* stream) {
   if (!code) return fail(QUOKA_ERR_INVALID_ARG, "code is NULL");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -118,3 +118,18 @@ def test_null_shape_rejected():
                             Bd._host_i32((0,)), 1, FAKE, None, FAKE, 1 << 20, None) == \
         Bd.QUOKA_ERR_INVALID_ARG
     assert "NULL" in lib.quoka_last_error().decode()
+
+
+@no_gpu
+def test_noalloc_rejects_oversize_before_launch():
+    """A call whose scratch would not fit the built-in array is refused host-side."""
+    lib = Bd.lib()
+    shape = Bd.QuokaShape(64, 64, 8, 128, 64, Bd.QUOKA_BF16)
+    need = lib.quoka_select_workspace_size(ctypes.byref(shape), 0, 64)
+    assert need > (32 << 20)
+    st = lib.quoka_select_noalloc(ctypes.byref(shape), FAKE, FAKE,
+                                  Bd._host_i64([0] + [64 * (i + 1) for i in range(64)]),
+                                  Bd._host_i32([0] * 64), 64, Bd._host_i32([1] * 64), 1, FAKE,
+                                  None, None)
+    assert st == Bd.QUOKA_ERR_WORKSPACE
+    assert "built-in scratch" in lib.quoka_last_error().decode()
