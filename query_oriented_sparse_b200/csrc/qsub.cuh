@@ -8,7 +8,9 @@
 // slab (L2-resident) for c_t = cos(q_t, mean).  A 4-pass block radix select finds the
 // Nk-th smallest orderable key, then a scan keeps, in ascending t, every query below
 // it plus the lowest-index ties.  The kept rows are copied (raw values) into the
-// per-KV-head operand block used by the scoring GEMM, with their fp32 1/|q|.
+// per-KV-head operand block used by the scoring GEMM, with their fp32 1/|q| and a
+// column bias; each head's block is padded to nkp rows (a multiple of 16) with zero
+// rows whose bias is -inf, so a padded column can never win the max pooling.
 #pragma once
 #include "common.cuh"
 
@@ -73,8 +75,9 @@ __device__ __forceinline__ uint32_t block_radix_select_smallest(const uint32_t* 
 
 template <typename T, int D>
 __global__ void __launch_bounds__(QSUB_THREADS)
-qsub_kernel(const T* __restrict__ q, int h_q, int C, int nk, int nq,
-            int32_t* __restrict__ kept_out, T* __restrict__ qsel, float* __restrict__ qinv) {
+qsub_kernel(const T* __restrict__ q, int h_q, int C, int nk, int nkp, int nq,
+            int32_t* __restrict__ kept_out, T* __restrict__ qsel, float* __restrict__ qinv,
+            float* __restrict__ qbias) {
   constexpr int PER = D / 32;                 // elements per lane per row
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* inv = reinterpret_cast<float*>(smem_raw);
@@ -167,21 +170,22 @@ qsub_kernel(const T* __restrict__ q, int h_q, int C, int nk, int nq,
   }
   __syncthreads();
 
-  // outputs: kept positions, 1/|q| and the raw kept rows
-  const size_t row0 = (size_t)bh * nk;        // == ((b*h_kv + g)*G + h%G) * nk
-  for (int i = tid; i < nk; i += blockDim.x) {
-    const int t = sel_t[i];
-    qinv[row0 + i] = inv[t];
-    if (kept_out) kept_out[(size_t)bh * nq + i] = t;
+  // outputs: kept positions, 1/|q|, column bias and the raw kept rows (padded to nkp)
+  const size_t row0 = (size_t)bh * nkp;       // == ((b*h_kv + g)*G + h%G) * nkp
+  for (int i = tid; i < nkp; i += blockDim.x) {
+    const bool real = i < nk;
+    qinv[row0 + i] = real ? inv[sel_t[i]] : 0.f;
+    qbias[row0 + i] = real ? 0.f : -INFINITY;
+    if (kept_out && i < nq) kept_out[(size_t)bh * nq + i] = real ? sel_t[i] : -1;
   }
   if (kept_out)
-    for (int i = nk + tid; i < nq; i += blockDim.x) kept_out[(size_t)bh * nq + i] = -1;
+    for (int i = nkp + tid; i < nq; i += blockDim.x) kept_out[(size_t)bh * nq + i] = -1;
   constexpr int VEC = 16 / sizeof(T);          // elements per 16-byte vector
   constexpr int NV = D / VEC;                  // vectors per row
-  for (int e = tid; e < nk * NV; e += blockDim.x) {
+  for (int e = tid; e < nkp * NV; e += blockDim.x) {
     const int i = e / NV, v = e % NV;
-    const int t = sel_t[i];
-    const uint4 val = __ldg(reinterpret_cast<const uint4*>(qh + (size_t)t * D) + v);
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (i < nk) val = __ldg(reinterpret_cast<const uint4*>(qh + (size_t)sel_t[i] * D) + v);
     reinterpret_cast<uint4*>(qsel + (row0 + i) * D)[v] = val;
   }
 }

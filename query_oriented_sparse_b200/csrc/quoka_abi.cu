@@ -1,6 +1,7 @@
 // Host side of libquoka.so: argument validation, workspace layout and kernel launches
 // behind the C ABI declared in include/quoka.h.  Every check runs before any CUDA
 // call, so an invalid call launches nothing.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <map>
@@ -11,6 +12,7 @@
 #include "common.cuh"
 #include "qsub.cuh"
 #include "score_simt.cuh"
+#include "score_tc.cuh"
 #include "topk.cuh"
 #include "attn_simt.cuh"
 
@@ -99,24 +101,84 @@ quoka_status build_table(const Dims& d, const int64_t* kv_off, const int32_t* pr
 }
 
 struct WsLayout {
-  size_t qsel, qinv, pooled, total;
+  size_t qsel, qinv, qbias, pooled, total;
   long long pooled_stride;  // floats per (sequence, KV head) row
-  int nk;
+  long long cg_stride;      // floats between column-group partial arrays
+  int nk, nkp;              // kept queries per head, and that count padded to 16
+  int ncg, heads_per_cg;    // column groups per KV head for the tensor-core scoring
+  bool tc;                  // tensor-core scoring (bf16) or CUDA-core scoring (fp32)
 };
 
 WsLayout ws_layout(const Dims& d, int max_prefix, int nq) {
   WsLayout w;
   w.nk = nq < d.C ? nq : d.C;
+  w.nkp = (w.nk + 15) / 16 * 16;
+  w.tc = d.dt == QUOKA_BF16 && w.nkp <= STC_MAXCOLS;
+  if (w.tc) {
+    const int hmax = STC_MAXCOLS / w.nkp;
+    w.ncg = (d.G + hmax - 1) / hmax;
+    w.heads_per_cg = (d.G + w.ncg - 1) / w.ncg;
+  } else {
+    w.ncg = 1;
+    w.heads_per_cg = d.G;
+  }
+  const size_t rows = (size_t)d.batch * d.h_q * w.nkp;
   size_t off = 0;
   w.qsel = off;
-  off = align_up(off + (size_t)d.batch * d.h_q * w.nk * d.D * d.esz, 256);
+  off = align_up(off + rows * d.D * d.esz, 256);
   w.qinv = off;
-  off = align_up(off + (size_t)d.batch * d.h_q * w.nk * 4, 256);
+  off = align_up(off + rows * 4, 256);
+  w.qbias = off;
+  off = align_up(off + rows * 4, 256);
   w.pooled_stride = (long long)align_up((size_t)(max_prefix > 0 ? max_prefix : 1), 128);
+  w.cg_stride = (long long)d.batch * d.h_kv * w.pooled_stride;
   w.pooled = off;
-  off = align_up(off + (size_t)d.batch * d.h_kv * w.pooled_stride * 4, 256);
+  off = align_up(off + (size_t)w.ncg * w.cg_stride * 4, 256);
   w.total = off;
   return w;
+}
+
+// ---- TMA tensor maps (driver entry point fetched through the runtime) ----------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// Row-major [rows, cols] bf16 matrix, box of box_cols x box_rows, 128-byte swizzle.
+quoka_status make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                           uint32_t box_cols, uint32_t box_rows, const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(QUOKA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  if (rows >= (1ull << 31)) return fail(QUOKA_ERR_UNSUPPORTED, "%s has more than 2^31 rows", what);
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QUOKA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed: %d", what, (int)r);
+  return QUOKA_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
 }
 
 // Raises a kernel's dynamic shared-memory limit, once per (kernel, device).
@@ -137,33 +199,78 @@ cudaError_t ensure_smem(K kernel, int bytes) {
   return e;
 }
 
+template <int D>
+quoka_status launch_score_tc(const Dims& d, const SeqTable& tab, long long rows, const void* k,
+                             unsigned char* ws, const WsLayout& w, cudaStream_t st) {
+  ScoreTcParams p;
+  p.h_kv = d.h_kv;
+  p.G = d.G;
+  p.nkp = w.nkp;
+  p.ncg = w.ncg;
+  p.heads_per_cg = w.heads_per_cg;
+  p.rows_per_head = rows;
+  p.pooled_stride = w.pooled_stride;
+  p.cg_stride = w.cg_stride;
+  p.inv_G = 1.0f / (float)d.G;
+  long long units = 0;
+  for (int b = 0; b < d.batch; ++b) {
+    p.unit_base[b] = (int)units;
+    units += (long long)d.h_kv * w.ncg * ((tab.prefix[b] + STC_BM - 1) / STC_BM);
+  }
+  for (int b = d.batch; b <= QUOKA_MAX_BATCH; ++b) p.unit_base[b] = (int)units;
+  if (units == 0) return QUOKA_OK;
+  if (units >= (1ll << 31)) return fail(QUOKA_ERR_UNSUPPORTED, "too many key tiles");
+  p.total_units = (int)units;
+  CUtensorMap kmap, qmap;
+  quoka_status s;
+  if ((s = make_map_bf16(&kmap, k, (uint64_t)d.h_kv * rows, D, 64, STC_BM, "k_cache")) != QUOKA_OK) return s;
+  if ((s = make_map_bf16(&qmap, ws + w.qsel, (uint64_t)d.batch * d.h_q * w.nkp, D, 64, STC_QBOX,
+                         "kept queries")) != QUOKA_OK)
+    return s;
+  cudaError_t e;
+  const int smem = StcCfg<D>::SMEM;
+  if ((e = ensure_smem(score_tc_kernel<D>, smem)) != cudaSuccess) return cuda_fail(e, "score_tc smem");
+  const int grid = (int)std::min<long long>(units, sm_count());
+  score_tc_kernel<D><<<grid, STC_THREADS, smem, st>>>(
+      kmap, qmap, tab, p, reinterpret_cast<const float*>(ws + w.qinv),
+      reinterpret_cast<const float*>(ws + w.qbias), reinterpret_cast<float*>(ws + w.pooled));
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score_tc launch");
+  return QUOKA_OK;
+}
+
 template <typename T, int D>
 quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                            const void* k, int nq, int b_max, int32_t* idx_out, int32_t* kept_out,
                            unsigned char* ws, const WsLayout& w, cudaStream_t st) {
   T* qsel = reinterpret_cast<T*>(ws + w.qsel);
   float* qinv = reinterpret_cast<float*>(ws + w.qinv);
+  float* qbias = reinterpret_cast<float*>(ws + w.qbias);
   float* pooled = reinterpret_cast<float*>(ws + w.pooled);
   cudaError_t e;
 
   const int s1 = qsub_smem_bytes<D>(d.C);
   if ((e = ensure_smem(qsub_kernel<T, D>, s1)) != cudaSuccess) return cuda_fail(e, "qsub smem");
   qsub_kernel<T, D><<<d.batch * d.h_q, QSUB_THREADS, s1, st>>>(
-      reinterpret_cast<const T*>(q), d.h_q, d.C, w.nk, nq, kept_out, qsel, qinv);
+      reinterpret_cast<const T*>(q), d.h_q, d.C, w.nk, w.nkp, nq, kept_out, qsel, qinv, qbias);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "qsub launch");
 
   if (tab.max_prefix > 0) {
-    const int s2 = score_simt_smem_bytes<D>(d.G);
-    if ((e = ensure_smem(score_simt_kernel<T, D>, s2)) != cudaSuccess) return cuda_fail(e, "score smem");
-    dim3 grid((tab.max_prefix + SCS_KEYS - 1) / SCS_KEYS, d.h_kv, d.batch);
-    score_simt_kernel<T, D><<<grid, SCS_THREADS, s2, st>>>(
-        reinterpret_cast<const T*>(k), rows, tab, d.h_kv, d.G, w.nk, qsel, qinv, pooled,
-        w.pooled_stride);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score launch");
+    if (w.tc) {
+      quoka_status s = launch_score_tc<D>(d, tab, rows, k, ws, w, st);
+      if (s != QUOKA_OK) return s;
+    } else {
+      const int s2 = score_simt_smem_bytes<D>(d.G);
+      if ((e = ensure_smem(score_simt_kernel<T, D>, s2)) != cudaSuccess) return cuda_fail(e, "score smem");
+      dim3 grid((tab.max_prefix + SCS_KEYS - 1) / SCS_KEYS, d.h_kv, d.batch);
+      score_simt_kernel<T, D><<<grid, SCS_THREADS, s2, st>>>(
+          reinterpret_cast<const T*>(k), rows, tab, d.h_kv, d.G, w.nkp, qsel, qinv, qbias, pooled,
+          w.pooled_stride);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score launch");
+    }
   }
 
-  topk_kernel<<<d.batch * d.h_kv * TOPK_CS, TOPK_THREADS, 0, st>>>(pooled, w.pooled_stride, tab,
-                                                                   d.h_kv, b_max, idx_out);
+  topk_kernel<<<d.batch * d.h_kv * TOPK_CS, TOPK_THREADS, 0, st>>>(
+      pooled, w.pooled_stride, w.ncg, w.cg_stride, 1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
   return QUOKA_OK;
 }

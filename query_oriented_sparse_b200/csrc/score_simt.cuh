@@ -22,15 +22,16 @@ constexpr int SCS_THREADS = 256;
 template <int D>
 __host__ __device__ constexpr int score_simt_smem_bytes(int G) {
   return (SCS_KEYS * (D + 1) + SCS_QROWS * (D + 1) + SCS_KEYS * (SCS_QROWS + 1) +
-          SCS_KEYS * G + SCS_KEYS + SCS_QROWS) * 4;
+          SCS_KEYS * G + SCS_KEYS + 2 * SCS_QROWS) * 4;
 }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(SCS_THREADS)
 score_simt_kernel(const T* __restrict__ k_cache, long long rows_per_head,
-                  const __grid_constant__ SeqTable tab, int h_kv, int G, int nk,
+                  const __grid_constant__ SeqTable tab, int h_kv, int G, int nkp,
                   const T* __restrict__ qsel, const float* __restrict__ qinv,
-                  float* __restrict__ pooled, long long pooled_stride) {
+                  const float* __restrict__ qbias, float* __restrict__ pooled,
+                  long long pooled_stride) {
   constexpr int LD = D + 1;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* Ks = reinterpret_cast<float*>(smem_raw);
@@ -39,15 +40,17 @@ score_simt_kernel(const T* __restrict__ k_cache, long long rows_per_head,
   float* mx = Sb + SCS_KEYS * (SCS_QROWS + 1);   // [64 keys][G]
   float* knorm = mx + SCS_KEYS * G;
   float* qiv = knorm + SCS_KEYS;
+  float* qbs = qiv + SCS_QROWS;
 
   const int b = blockIdx.z, g = blockIdx.y, j0 = blockIdx.x * SCS_KEYS;
   const int P = tab.prefix[b];
   if (j0 >= P) return;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const T* kbase = k_cache + ((size_t)g * rows_per_head + tab.kv_off[b]) * D;
-  const int nrows = G * nk;
+  const int nrows = G * nkp;
   const T* qbase = qsel + (size_t)(b * h_kv + g) * nrows * D;
   const float* ibase = qinv + (size_t)(b * h_kv + g) * nrows;
+  const float* bbase = qbias + (size_t)(b * h_kv + g) * nrows;
 
   // stage the key tile (zeros past P) and reset the running maxima
   for (int e = tid * 4; e < SCS_KEYS * D; e += SCS_THREADS * 4) {
@@ -74,7 +77,10 @@ score_simt_kernel(const T* __restrict__ k_cache, long long rows_per_head,
 #pragma unroll
       for (int i = 0; i < 4; ++i) Qs[r * LD + c + i] = x[i];
     }
-    if (tid < SCS_QROWS) qiv[tid] = (q0 + tid < nrows) ? ibase[q0 + tid] : 0.f;
+    if (tid < SCS_QROWS) {
+      qiv[tid] = (q0 + tid < nrows) ? ibase[q0 + tid] : 0.f;
+      qbs[tid] = (q0 + tid < nrows) ? bbase[q0 + tid] : -INFINITY;
+    }
     __syncthreads();
 
     float acc[4][4];
@@ -98,12 +104,13 @@ score_simt_kernel(const T* __restrict__ k_cache, long long rows_per_head,
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        Sb[(ty + 16 * i) * (SCS_QROWS + 1) + tx + 16 * j] = acc[i][j] * qiv[tx + 16 * j];
+        Sb[(ty + 16 * i) * (SCS_QROWS + 1) + tx + 16 * j] =
+            fmaf(acc[i][j], qiv[tx + 16 * j], qbs[tx + 16 * j]);
     __syncthreads();
     if (tid < SCS_KEYS) {
       const int lim = min(SCS_QROWS, nrows - q0);
       for (int c = 0; c < lim; ++c) {
-        const int hl = (q0 + c) / nk;
+        const int hl = (q0 + c) / nkp;
         const float v = Sb[tid * (SCS_QROWS + 1) + c];
         float* m = &mx[tid * G + hl];
         *m = fmaxf(*m, v);

@@ -10,6 +10,8 @@
 // the same digit decision.  Keys above T are kept, plus the lowest-index keys equal
 // to T; a cluster exchange of per-slice counts and block scans give each kept index
 // its output slot, so the result is deterministic and sorted without a sort.
+// When the scoring kernel split a KV head's kept queries into several column groups,
+// a first pass adds the groups' partial sums (in group order) and applies 1/G.
 #pragma once
 #include <cooperative_groups.h>
 #include "common.cuh"
@@ -22,8 +24,8 @@ constexpr int TOPK_CS = 8;
 constexpr int TOPK_THREADS = 512;
 
 __global__ void __cluster_dims__(TOPK_CS, 1, 1) __launch_bounds__(TOPK_THREADS)
-topk_kernel(const float* __restrict__ pooled, long long pooled_stride,
-            const __grid_constant__ SeqTable tab, int h_kv, int b_max,
+topk_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, long long cg_stride,
+            float inv_G, const __grid_constant__ SeqTable tab, int h_kv, int b_max,
             int32_t* __restrict__ idx_out) {
   cg::cluster_group cluster = cg::this_cluster();
   __shared__ int hist[2][256];
@@ -38,8 +40,18 @@ topk_kernel(const float* __restrict__ pooled, long long pooled_stride,
   const int P = tab.prefix[b], B = tab.nsel[b];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* out = idx_out + (size_t)head * b_max;
-  const float* sc = pooled + (size_t)head * pooled_stride;
+  float* sc = pooled + (size_t)head * pooled_stride;
   const int stride = TOPK_CS * blockDim.x;
+
+  if (ncg > 1) {                               // sum the column groups' partial scores
+    for (int j = rank * blockDim.x + threadIdx.x; j < P; j += stride) {
+      float s = sc[j];
+      for (int c = 1; c < ncg; ++c) s += sc[c * cg_stride + j];
+      sc[j] = s * inv_G;
+    }
+    __threadfence();
+    cluster.sync();
+  }
 
   for (int i = B + rank * blockDim.x + tid; i < b_max; i += stride) out[i] = -1;
   if (B >= P) {                                // keep every prefix key (P == 0 included)
@@ -59,7 +71,7 @@ topk_kernel(const float* __restrict__ pooled, long long pooled_stride,
     for (int i = tid; i < 256; i += blockDim.x) hcur[i] = 0;
     __syncthreads();
     for (int j = lo + tid; j < hi; j += blockDim.x) {
-      const uint32_t key = float_to_ordered(__ldg(sc + j));
+      const uint32_t key = float_to_ordered(sc[j]);
       if ((key & mask) == prefix) atomicAdd(&hcur[(key >> shift) & 255u], 1);
     }
     cluster.sync();
@@ -104,7 +116,7 @@ topk_kernel(const float* __restrict__ pooled, long long pooled_stride,
   // per-slice counts of keys above / equal to the threshold
   int c_gt = 0, c_eq = 0;
   for (int j = lo + tid; j < hi; j += blockDim.x) {
-    const uint32_t key = float_to_ordered(__ldg(sc + j));
+    const uint32_t key = float_to_ordered(sc[j]);
     c_gt += key > thr;
     c_eq += key == thr;
   }
@@ -130,7 +142,7 @@ topk_kernel(const float* __restrict__ pooled, long long pooled_stride,
   for (int base = lo; base < hi; base += blockDim.x) {
     const int j = base + tid;
     const bool valid = j < hi;
-    const uint32_t key = valid ? float_to_ordered(__ldg(sc + j)) : 0u;
+    const uint32_t key = valid ? float_to_ordered(sc[j]) : 0u;
     const int is_eq = (valid && key == thr) ? 1 : 0;
     int tot_eq;
     const int eq_rank = block_exclusive_scan(is_eq, scan_scratch, &tot_eq) + run_eq;
