@@ -1,0 +1,353 @@
+// K4 (tensor-core form, bf16): dense attention of the chunk over its compacted cache
+// (QUOKA page, Figure 1(a): the sub-selected KV cache goes into a dense attention
+// kernel; QUILT page: the K/V entries a group of queries selected in common are loaded
+// once and reused by all of them).
+//
+// One CTA per (sequence, KV head, 2 x TP chunk positions).  Its two 128-row query
+// tiles pack the G query heads of the KV head (TP = 128 / G positions each), so every
+// gathered K/V tile in shared memory feeds 256 query rows of G heads.  K/V rows are
+// gathered straight from the cache by TMA (tile::gather4, four rows per instruction,
+// 128-byte swizzle) using the selected indices, followed by the chunk's own rows.
+//
+// TMEM holds S0, S1 (128 x 128 fp32 logits of each tile) and O0, O1 (128 x d fp32).
+// Warp 0 loads, one thread of warp 1 issues tcgen05.mma, warps 2-5 and 6-9 run the
+// softmax of tile 0 and tile 1 (one thread per query row) so that one tile's
+// exponentials overlap the other tile's MMAs.  P is written back as bf16 over the
+// first 64 columns of S and consumed from TMEM by the P.V MMA (A operand in TMEM).
+// The online softmax keeps its running max per row in fp32 and rescales O in TMEM
+// only when the max grows by more than 2^8, so the exponent stays bounded.
+#pragma once
+#include "tc_ptx.cuh"
+
+namespace quoka {
+
+constexpr int ATC_THREADS = 320;   // warp 0 load, warp 1 MMA, 2-5 softmax tile 0, 6-9 tile 1
+constexpr int ATC_KST = 2;         // K stages
+constexpr int ATC_VST = 2;         // V stages
+constexpr float ATC_RESCALE_LOG2 = 8.0f;
+
+struct AttnTcParams {
+  int h_q, h_kv, G, C, TP, b_max;
+  long long rows_per_head;
+  float scale_log2;                // log2(e) / sqrt(d)
+};
+
+template <int D>
+struct AtcCfg {
+  static constexpr int KB = D / 64;
+  static constexpr int TILE_BYTES = 128 * D * 2;  // 128 rows of one operand
+  static constexpr int Q_BYTES = 2 * TILE_BYTES;
+  static constexpr int K_BYTES = ATC_KST * TILE_BYTES;
+  static constexpr int V_BYTES = ATC_VST * TILE_BYTES;
+  static constexpr int NBAR = 1 + 2 * ATC_KST + 2 * ATC_VST + 2 + 2 + 2;
+  static constexpr int SMEM = 1024 + Q_BYTES + K_BYTES + V_BYTES + NBAR * 8 + 16;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int D>
+__global__ void __launch_bounds__(ATC_THREADS, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+               const __grid_constant__ CUtensorMap vmap, const __grid_constant__ SeqTable tab,
+               const __grid_constant__ AttnTcParams p, const int32_t* __restrict__ idx,
+               __nv_bfloat16* __restrict__ out) {
+  using Cfg = AtcCfg<D>;
+  constexpr int KB = Cfg::KB;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + Cfg::Q_BYTES;
+  uint8_t* sV = sK + Cfg::K_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + Cfg::V_BYTES);
+  uint64_t* qfull = bars;
+  uint64_t* kfull = bars + 1;
+  uint64_t* kempty = kfull + ATC_KST;
+  uint64_t* vfull = kempty + ATC_KST;
+  uint64_t* vempty = vfull + ATC_VST;
+  uint64_t* sfull = vempty + ATC_VST;   // [2]
+  uint64_t* pready = sfull + 2;         // [2]
+  uint64_t* odone = pready + 2;         // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(odone + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.z, g = blockIdx.y;
+  const int npairs = (p.C + 2 * p.TP - 1) / (2 * p.TP);
+  const int pair = npairs - 1 - (int)blockIdx.x;           // longest key ranges first
+  const int t0 = pair * 2 * p.TP;
+  const int P = tab.prefix[b], nsel = tab.nsel[b];
+  const int tend = min(p.C, t0 + 2 * p.TP);                  // positions [t0, tend)
+  const int nkeys = nsel + tend;                             // selected + chunk keys 0..tend-1
+  const int nblk = (nkeys + 127) / 128;
+  const long long seq_row0 = (long long)g * p.rows_per_head + tab.kv_off[b];
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(qfull, 1);
+    for (int s = 0; s < ATC_KST; ++s) { ptx::mbar_init(&kfull[s], 1); ptx::mbar_init(&kempty[s], 1); }
+    for (int s = 0; s < ATC_VST; ++s) { ptx::mbar_init(&vfull[s], 1); ptx::mbar_init(&vempty[s], 1); }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&sfull[i], 1);
+      ptx::mbar_init(&pready[i], 4);
+      ptx::mbar_init(&odone[i], 1);
+    }
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- loads: Q once, then K and V blocks by gather4 ----------------
+    if (lane == 0) {
+      ptx::prefetch_tmap(&qmap);
+      ptx::prefetch_tmap(&kmap);
+      ptx::prefetch_tmap(&vmap);
+    }
+    const int32_t* sel = idx + (size_t)(b * p.h_kv + g) * p.b_max;
+    // Q: 2 tiles x 32 groups of 4 rows; row r of tile i is head r / TP, position
+    // t0 + i*TP + r % TP (rows past G*TP or C repeat a valid row; never stored)
+    if (lane == 0) ptx::mbar_expect_tx(qfull, (uint32_t)Cfg::Q_BYTES);
+    __syncwarp();
+    for (int grp = lane; grp < 64; grp += 32) {
+      const int tile = grp >> 5, r0 = (grp & 31) * 4;
+      int rows[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r = r0 + k;
+        int hl = r / p.TP, t = t0 + tile * p.TP + r % p.TP;
+        if (hl >= p.G || t >= p.C) { hl = 0; t = t0; }
+        rows[k] = (b * p.h_q + g * p.G + hl) * p.C + t;
+      }
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb)
+        ptx::tma_gather4(sQ + tile * Cfg::TILE_BYTES + kb * 16384 + r0 * 128, &qmap, qfull, kb * 64,
+                         rows[0], rows[1], rows[2], rows[3]);
+    }
+    bool ok = true;
+    for (int j = 0; j < nblk && ok; ++j) {
+      int rows[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int kk = j * 128 + lane * 4 + k;
+        int r;
+        if (kk < nsel) {
+          r = sel[kk];
+          if (r < 0 || r >= P) { flag_error(ERR_BAD_INDEX); r = P; }
+        } else if (kk < nkeys) {
+          r = P + (kk - nsel);
+        } else {
+          r = P;                                   // padding key, masked in the softmax
+        }
+        rows[k] = (int)(seq_row0 + r);
+      }
+      const int ks = j % ATC_KST, vs = j % ATC_VST;
+      const uint32_t kph = (uint32_t)(j / ATC_KST) & 1u, vph = (uint32_t)(j / ATC_VST) & 1u;
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&kempty[ks], kph ^ 1u));
+      if (!ok) break;
+      if (lane == 0) ptx::mbar_expect_tx(&kfull[ks], (uint32_t)Cfg::TILE_BYTES);
+      __syncwarp();
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb)
+        ptx::tma_gather4(sK + ks * Cfg::TILE_BYTES + kb * 16384 + lane * 512, &kmap, &kfull[ks],
+                         kb * 64, rows[0], rows[1], rows[2], rows[3]);
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&vempty[vs], vph ^ 1u));
+      if (!ok) break;
+      if (lane == 0) ptx::mbar_expect_tx(&vfull[vs], (uint32_t)Cfg::TILE_BYTES);
+      __syncwarp();
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb)
+        ptx::tma_gather4(sV + vs * Cfg::TILE_BYTES + kb * 16384 + lane * 512, &vmap, &vfull[vs],
+                         kb * 64, rows[0], rows[1], rows[2], rows[3]);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc_s = ptx::idesc_bf16(128, 128, false);
+      const uint32_t idesc_o = ptx::idesc_bf16(128, D, true);
+      bool ok = ptx::mbar_wait(qfull, 0);
+      auto issue_s = [&](int i, int j) {
+        const int ks = j % ATC_KST;
+        const uint32_t a0 = ptx::smem_u32(sQ + i * Cfg::TILE_BYTES);
+        const uint32_t b0 = ptx::smem_u32(sK + ks * Cfg::TILE_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            ptx::mma_bf16_ss(tmem + (uint32_t)(i * 128),
+                             ptx::sdesc_sw128(a0 + kb * 16384 + k * 32, 16, 1024),
+                             ptx::sdesc_sw128(b0 + kb * 16384 + k * 32, 16, 1024), idesc_s,
+                             (kb | k) ? 1u : 0u);
+        ptx::tc_commit(&sfull[i]);
+      };
+      auto issue_pv = [&](int i, int j) {
+        const int vs = j % ATC_VST;
+        const uint32_t b0 = ptx::smem_u32(sV + vs * Cfg::TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)                          // 16 keys per MMA
+          ptx::mma_bf16_ts(tmem + (uint32_t)(256 + i * 128), tmem + (uint32_t)(i * 128 + k * 8),
+                           ptx::sdesc_sw128(b0 + k * 2048, 16384, 1024), idesc_o,
+                           (j > 0 || k > 0) ? 1u : 0u);
+        ptx::tc_commit(&odone[i]);
+      };
+      if (ok) ok = ptx::mbar_wait(&kfull[0], 0);
+      if (ok) {
+        ptx::tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        ptx::tc_commit(&kempty[0]);
+      }
+      for (int j = 0; j < nblk && ok; ++j) {
+        const uint32_t par = (uint32_t)j & 1u;
+        ok = ptx::mbar_wait(&vfull[j % ATC_VST], (uint32_t)(j / ATC_VST) & 1u);
+        if (ok) ok = ptx::mbar_wait(&pready[0], par);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_pv(0, j);
+        const bool more = j + 1 < nblk;
+        if (more) {
+          ok = ptx::mbar_wait(&kfull[(j + 1) % ATC_KST], (uint32_t)((j + 1) / ATC_KST) & 1u);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        ok = ptx::mbar_wait(&pready[1], par);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_pv(1, j);
+        ptx::tc_commit(&vempty[j % ATC_VST]);
+        if (more) {
+          issue_s(1, j + 1);
+          ptx::tc_commit(&kempty[(j + 1) % ATC_KST]);
+        }
+      }
+    }
+  } else {
+    // ---------------- softmax: warps 2-5 tile 0, warps 6-9 tile 1 ----------------
+    const int tile = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                      // row of the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + (uint32_t)(tile * 128);
+    const uint32_t o_addr = tmem + lane_off + (uint32_t)(256 + tile * 128);
+    const int hl = r / p.TP;
+    const int t = t0 + tile * p.TP + r % p.TP;
+    const bool row_valid = hl < p.G && t < p.C;
+    const int tmin = t0 + tile * p.TP;                      // smallest position in this tile
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nblk && ok; ++j) {
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&sfull[tile], (uint32_t)j & 1u));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 128; c += 32) {
+        uint32_t u[32];
+        ptx::tmem_ld32(s_addr + (uint32_t)c, u);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(u[i]);
+      }
+      ptx::tmem_ld_wait();
+      const int kb0 = j * 128;
+      if (kb0 + 127 >= nsel + tmin || kb0 + 127 >= nkeys) {  // block reaches the causal part
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int kk = kb0 + c;
+          const bool valid = kk < nkeys && (kk < nsel || kk - nsel <= t);
+          if (!valid) s[c] = -INFINITY;
+        }
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      const float m_cand = mx * p.scale_log2;
+      const bool grow = m_cand > m_run + ATC_RESCALE_LOG2 || (m_run == -INFINITY && m_cand > -INFINITY);
+      float alpha = 1.f;
+      if (grow) {
+        alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_cand);
+        m_run = m_cand;
+        l_run *= alpha;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O holds blocks 0..j-1 once the previous P.V of this tile has finished
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&odone[tile], (uint32_t)(j - 1) & 1u));
+        if (!ok) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D; c += 16) {
+          uint32_t u[16];
+          ptx::tmem_ld16(o_addr + (uint32_t)c, u);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          ptx::tmem_st16(o_addr + (uint32_t)c, u);
+        }
+        ptx::tmem_st_wait();
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; c += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = exp2f(fmaf(s[c + 2 * i], p.scale_log2, -m_use));
+          const float p1 = exp2f(fmaf(s[c + 2 * i + 1], p.scale_log2, -m_use));
+          lsum += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        ptx::tmem_st16(s_addr + (uint32_t)(c / 2), pk);
+      }
+      ptx::tmem_st_wait();
+      l_run += lsum;
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&pready[tile]);
+    }
+    // epilogue: O / l -> bf16 rows of out[b, g*G + hl, t, :]
+    if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&odone[tile], (uint32_t)(nblk - 1) & 1u));
+    if (ok) {
+      ptx::tc_fence_after();
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      __nv_bfloat16* orow = out + ((size_t)(b * p.h_q + g * p.G + (row_valid ? hl : 0)) * p.C +
+                                   (row_valid ? t : 0)) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 16) {
+        uint32_t u[16];
+        ptx::tmem_ld16(o_addr + (uint32_t)c, u);
+        ptx::tmem_ld_wait();
+        uint4 w0, w1;
+        w0.x = pack_bf16(__uint_as_float(u[0]) * inv_l, __uint_as_float(u[1]) * inv_l);
+        w0.y = pack_bf16(__uint_as_float(u[2]) * inv_l, __uint_as_float(u[3]) * inv_l);
+        w0.z = pack_bf16(__uint_as_float(u[4]) * inv_l, __uint_as_float(u[5]) * inv_l);
+        w0.w = pack_bf16(__uint_as_float(u[6]) * inv_l, __uint_as_float(u[7]) * inv_l);
+        w1.x = pack_bf16(__uint_as_float(u[8]) * inv_l, __uint_as_float(u[9]) * inv_l);
+        w1.y = pack_bf16(__uint_as_float(u[10]) * inv_l, __uint_as_float(u[11]) * inv_l);
+        w1.z = pack_bf16(__uint_as_float(u[12]) * inv_l, __uint_as_float(u[13]) * inv_l);
+        w1.w = pack_bf16(__uint_as_float(u[14]) * inv_l, __uint_as_float(u[15]) * inv_l);
+        if (row_valid) {
+          reinterpret_cast<uint4*>(orow + c)[0] = w0;
+          reinterpret_cast<uint4*>(orow + c)[1] = w1;
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace quoka

@@ -15,6 +15,7 @@
 #include "score_tc.cuh"
 #include "topk.cuh"
 #include "attn_simt.cuh"
+#include "attn_tc.cuh"
 
 using namespace quoka;
 
@@ -275,10 +276,39 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
   return QUOKA_OK;
 }
 
+template <int D>
+quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                            const void* k, const void* v, const int32_t* idx, int b_max,
+                            void* out, cudaStream_t st) {
+  AttnTcParams p;
+  p.h_q = d.h_q;
+  p.h_kv = d.h_kv;
+  p.G = d.G;
+  p.C = d.C;
+  p.TP = 128 / d.G;
+  p.b_max = b_max;
+  p.rows_per_head = rows;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  CUtensorMap qmap, kmap, vmap;
+  quoka_status s;
+  if ((s = make_map_bf16(&qmap, q, (uint64_t)d.batch * d.h_q * d.C, D, 64, 1, "q_chunk")) != QUOKA_OK) return s;
+  if ((s = make_map_bf16(&kmap, k, (uint64_t)d.h_kv * rows, D, 64, 1, "k_cache")) != QUOKA_OK) return s;
+  if ((s = make_map_bf16(&vmap, v, (uint64_t)d.h_kv * rows, D, 64, 1, "v_cache")) != QUOKA_OK) return s;
+  cudaError_t e;
+  const int smem = AtcCfg<D>::SMEM;
+  if ((e = ensure_smem(attn_tc_kernel<D>, smem)) != cudaSuccess) return cuda_fail(e, "attn_tc smem");
+  dim3 grid((d.C + 2 * p.TP - 1) / (2 * p.TP), d.h_kv, d.batch);
+  attn_tc_kernel<D><<<grid, ATC_THREADS, smem, st>>>(qmap, kmap, vmap, tab, p, idx,
+                                                      reinterpret_cast<__nv_bfloat16*>(out));
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_tc launch");
+  return QUOKA_OK;
+}
+
 template <typename T, int D>
 quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                          const void* k, const void* v, const int32_t* idx, int b_max, void* out,
                          cudaStream_t st) {
+  if (d.dt == QUOKA_BF16) return launch_attn_tc<D>(d, tab, rows, q, k, v, idx, b_max, out, st);
   cudaError_t e;
   const int s = attn_simt_smem_bytes<D>();
   if ((e = ensure_smem(attn_simt_kernel<T, D>, s)) != cudaSuccess) return cuda_fail(e, "attn smem");
