@@ -35,7 +35,7 @@ from query_oriented_sparse_b200 import workloads as W  # noqa: E402
 METRIC = "chunked-prefill sparse-attn tokens/s (select+attend) and % of roofline, 1 B200"
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 4  # qsub, score, top-k, attention
+LAUNCHES_PER_STEP = 5  # qsub, score, top-k, compaction, attention
 
 
 def load_peaks():
@@ -234,6 +234,7 @@ def run_ours(args, w):
     ws = torch.empty(Bd.select_workspace_size(shape, max(w.prefix), w.nq), dtype=torch.uint8,
                      device=dev)
     idx = torch.empty(w.batch, w.h_kv, b_max, dtype=torch.int32, device=dev)
+    aws = torch.empty(max(Bd.attn_workspace_size(shape, b_max), 256), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -241,7 +242,7 @@ def run_ours(args, w):
     def step():
         Bd.quoka_select(q, k, t.kv_off, w.prefix, w.nq, w.budget, b_max, idx_out=idx,
                         workspace=ws)
-        Bd.sparse_chunk_attn(q, k, v, t.kv_off, w.prefix, w.budget, idx, out=out)
+        Bd.sparse_chunk_attn(q, k, v, t.kv_off, w.prefix, w.budget, idx, out=out, workspace=aws)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -262,7 +263,7 @@ def run_ours(args, w):
             Bd.quoka_select(q, k, t.kv_off, w.prefix, w.nq, w.budget, b_max, idx_out=idx,
                             workspace=ws)
             e1.record(stream)
-            Bd.sparse_chunk_attn(q, k, v, t.kv_off, w.prefix, w.budget, idx, out=out)
+            Bd.sparse_chunk_attn(q, k, v, t.kv_off, w.prefix, w.budget, idx, out=out, workspace=aws)
             e2.record(stream)
         torch.cuda.synchronize()
     if world > 1:

@@ -125,6 +125,9 @@ quoka_status quoka_select(const quoka_shape* shape, const void* q_chunk, const v
  * (QUOKA page, Figure 1(a): the compacted KV cache is fed to a dense attention
  * kernel; QUILT page: each shared K/V row is loaded once and reused by every query
  * that selected it - here the G query heads of a KV head share one selection).
+ * For bf16 the call first writes that compacted cache (per sequence and KV head: the
+ * selected rows, then the chunk's own rows) into `workspace`, then runs the dense
+ * kernel over it; fp32 gathers rows directly and needs no workspace.
  *
  * Query t of head h (KV head g = h / G) of sequence b attends to
  *     keys  { idx[b, g, i] : i < n_b }  U  { P + u : 0 <= u <= t }
@@ -137,14 +140,20 @@ quoka_status quoka_select(const quoka_shape* shape, const void* q_chunk, const v
  *   idx         device int32 [batch, h_kv, b_max], e.g. quoka_select's idx_out;
  *               entries [0, n_b) must be distinct prefix positions in [0, P)
  *   out         device [batch, h_q, chunk, head_dim]; must not alias an input
- * Errors: INVALID_ARG, UNSUPPORTED, CUDA.  idx entries are not range-checked on the
- * device; an entry outside [0, P) is a caller error.
+ *   workspace   device scratch of sparse_chunk_attn_workspace_size(shape, b_max)
+ *               bytes (may be NULL when that size is 0); contents on entry ignored
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.  An idx entry outside [0, P) is a
+ * caller error; the kernels substitute a valid row for it and set a bit in the device
+ * error word (quoka_device_error) instead of reading out of bounds.
  */
 quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk,
                                const void* k_cache, const void* v_cache,
                                const int64_t* kv_off, const int32_t* prefix_len,
                                const int32_t* budget, const int32_t* idx, int b_max,
-                               void* out, void* stream);
+                               void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device scratch sparse_chunk_attn() needs (0 for fp32; 0 if invalid). */
+size_t sparse_chunk_attn_workspace_size(const quoka_shape* shape, int b_max);
 
 /*
  * quoka_select_noalloc - quoka_select without a caller-provided workspace.

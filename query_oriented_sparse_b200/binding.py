@@ -43,7 +43,8 @@ SIGNATURES = {
     "quoka_select": (ctypes.c_int, [_SHAPE_P, _P, _P, _I64P, _I32P, ctypes.c_int, _I32P,
                                     ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "sparse_chunk_attn": (ctypes.c_int, [_SHAPE_P, _P, _P, _P, _I64P, _I32P, _I32P, _P,
-                                         ctypes.c_int, _P, _P]),
+                                         ctypes.c_int, _P, _P, ctypes.c_size_t, _P]),
+    "sparse_chunk_attn_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int]),
     "quoka_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "quoka_select_noalloc": (ctypes.c_int, [_SHAPE_P, _P, _P, _I64P, _I32P, ctypes.c_int, _I32P,
                                             ctypes.c_int, _P, _P, _P]),
@@ -175,18 +176,28 @@ def quoka_select_noalloc(q_chunk: torch.Tensor, k_cache: torch.Tensor, kv_off: S
     return idx_out
 
 
+def attn_workspace_size(shape: QuokaShape, b_max: int) -> int:
+    return int(lib().sparse_chunk_attn_workspace_size(ctypes.byref(shape), int(b_max)))
+
+
 def sparse_chunk_attn(q_chunk: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                       kv_off: Sequence[int], prefix_len: Sequence[int], budget: Sequence[int],
                       idx: torch.Tensor, out: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None,
                       stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """Attention of the chunk over its compacted cache; returns out [batch, h_q, C, d]."""
     shape = shape_of(q_chunk, k_cache)
     if out is None:
         out = torch.empty_like(q_chunk)
+    b_max = int(idx.shape[-1])
+    if workspace is None:
+        n = attn_workspace_size(shape, b_max)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q_chunk.device) if n else None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().sparse_chunk_attn(
         ctypes.byref(shape), _ptr(q_chunk), _ptr(k_cache), _ptr(v_cache), _host_i64(kv_off),
-        _host_i32(prefix_len), _host_i32(budget), _ptr(idx), int(idx.shape[-1]), _ptr(out),
-        ctypes.c_void_p(_stream(stream))))
+        _host_i32(prefix_len), _host_i32(budget), _ptr(idx), b_max, _ptr(out), _ptr(workspace),
+        ws_bytes, ctypes.c_void_p(_stream(stream))))
     return out
 
 

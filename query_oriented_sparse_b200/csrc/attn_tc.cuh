@@ -5,9 +5,11 @@
 //
 // One CTA per (sequence, KV head, 2 x TP chunk positions).  Its two 128-row query
 // tiles pack the G query heads of the KV head (TP = 128 / G positions each), so every
-// gathered K/V tile in shared memory feeds 256 query rows of G heads.  K/V rows are
-// gathered straight from the cache by TMA (tile::gather4, four rows per instruction,
-// 128-byte swizzle) using the selected indices, followed by the chunk's own rows.
+// K/V tile in shared memory feeds 256 query rows of G heads.  The query tiles are
+// gathered once by TMA (tile::gather4).  K/V come from the compacted cache of the
+// (sequence, KV head): the selected prefix rows followed by the chunk's own rows,
+// contiguous (compact.cuh), so one thread streams each 128-key block with two tiled
+// TMA loads per operand (128-byte swizzle) into a 3-stage K ring and a 2-stage V ring.
 //
 // TMEM holds S0, S1 (128 x 128 fp32 logits of each tile) and O0, O1 (128 x d fp32).
 // Warp 0 loads, one thread of warp 1 issues tcgen05.mma, warps 2-5 and 6-9 run the
@@ -22,12 +24,13 @@
 namespace quoka {
 
 constexpr int ATC_THREADS = 320;   // warp 0 load, warp 1 MMA, 2-5 softmax tile 0, 6-9 tile 1
-constexpr int ATC_KST = 2;         // K stages
+constexpr int ATC_KST = 3;         // K stages
 constexpr int ATC_VST = 2;         // V stages
 constexpr float ATC_RESCALE_LOG2 = 8.0f;
 
 struct AttnTcParams {
   int h_q, h_kv, G, C, TP, b_max;
+  long long kc_stride;             // rows per (sequence, KV head) block of the compacted cache
   long long rows_per_head;
   float scale_log2;                // log2(e) / sqrt(d)
 };
@@ -52,8 +55,7 @@ template <int D>
 __global__ void __launch_bounds__(ATC_THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap vmap, const __grid_constant__ SeqTable tab,
-               const __grid_constant__ AttnTcParams p, const int32_t* __restrict__ idx,
-               __nv_bfloat16* __restrict__ out) {
+               const __grid_constant__ AttnTcParams p, __nv_bfloat16* __restrict__ out) {
   using Cfg = AtcCfg<D>;
   constexpr int KB = Cfg::KB;
   extern __shared__ uint8_t smem_raw[];
@@ -82,7 +84,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   const int tend = min(p.C, t0 + 2 * p.TP);                  // positions [t0, tend)
   const int nkeys = nsel + tend;                             // selected + chunk keys 0..tend-1
   const int nblk = (nkeys + 127) / 128;
-  const long long seq_row0 = (long long)g * p.rows_per_head + tab.kv_off[b];
+  const int kc_row0 = (int)((long long)(b * p.h_kv + g) * p.kc_stride);
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(qfull, 1);
@@ -105,13 +107,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- loads: Q once, then K and V blocks by gather4 ----------------
+    // ---------------- loads: Q once by gather4, then K and V blocks by tiled TMA --------
     if (lane == 0) {
       ptx::prefetch_tmap(&qmap);
       ptx::prefetch_tmap(&kmap);
       ptx::prefetch_tmap(&vmap);
     }
-    const int32_t* sel = idx + (size_t)(b * p.h_kv + g) * p.b_max;
     // Q: 2 tiles x 32 groups of 4 rows; row r of tile i is head r / TP, position
     // t0 + i*TP + r % TP (rows past G*TP or C repeat a valid row; never stored)
     if (lane == 0) ptx::mbar_expect_tx(qfull, (uint32_t)Cfg::Q_BYTES);
@@ -131,41 +132,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         ptx::tma_gather4(sQ + tile * Cfg::TILE_BYTES + kb * 16384 + r0 * 128, &qmap, qfull, kb * 64,
                          rows[0], rows[1], rows[2], rows[3]);
     }
-    bool ok = true;
-    for (int j = 0; j < nblk && ok; ++j) {
-      int rows[4];
+    if (lane == 0) {
+      bool ok = true;
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int ks = j % ATC_KST, vs = j % ATC_VST;
+        const uint32_t kph = (uint32_t)(j / ATC_KST) & 1u, vph = (uint32_t)(j / ATC_VST) & 1u;
+        const int row = kc_row0 + j * 128;
+        ok = ptx::mbar_wait(&kempty[ks], kph ^ 1u);
+        if (!ok) break;
+        ptx::mbar_expect_tx(&kfull[ks], (uint32_t)Cfg::TILE_BYTES);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int kk = j * 128 + lane * 4 + k;
-        int r;
-        if (kk < nsel) {
-          r = sel[kk];
-          if (r < 0 || r >= P) { flag_error(ERR_BAD_INDEX); r = P; }
-        } else if (kk < nkeys) {
-          r = P + (kk - nsel);
-        } else {
-          r = P;                                   // padding key, masked in the softmax
-        }
-        rows[k] = (int)(seq_row0 + r);
+        for (int kb = 0; kb < KB; ++kb)
+          ptx::tma_load_2d(sK + ks * Cfg::TILE_BYTES + kb * 16384, &kmap, &kfull[ks], kb * 64, row);
+        ok = ptx::mbar_wait(&vempty[vs], vph ^ 1u);
+        if (!ok) break;
+        ptx::mbar_expect_tx(&vfull[vs], (uint32_t)Cfg::TILE_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+          ptx::tma_load_2d(sV + vs * Cfg::TILE_BYTES + kb * 16384, &vmap, &vfull[vs], kb * 64, row);
       }
-      const int ks = j % ATC_KST, vs = j % ATC_VST;
-      const uint32_t kph = (uint32_t)(j / ATC_KST) & 1u, vph = (uint32_t)(j / ATC_VST) & 1u;
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&kempty[ks], kph ^ 1u));
-      if (!ok) break;
-      if (lane == 0) ptx::mbar_expect_tx(&kfull[ks], (uint32_t)Cfg::TILE_BYTES);
-      __syncwarp();
-#pragma unroll
-      for (int kb = 0; kb < KB; ++kb)
-        ptx::tma_gather4(sK + ks * Cfg::TILE_BYTES + kb * 16384 + lane * 512, &kmap, &kfull[ks],
-                         kb * 64, rows[0], rows[1], rows[2], rows[3]);
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&vempty[vs], vph ^ 1u));
-      if (!ok) break;
-      if (lane == 0) ptx::mbar_expect_tx(&vfull[vs], (uint32_t)Cfg::TILE_BYTES);
-      __syncwarp();
-#pragma unroll
-      for (int kb = 0; kb < KB; ++kb)
-        ptx::tma_gather4(sV + vs * Cfg::TILE_BYTES + kb * 16384 + lane * 512, &vmap, &vfull[vs],
-                         kb * 64, rows[0], rows[1], rows[2], rows[3]);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -265,14 +250,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           if (!valid) s[c] = -INFINITY;
         }
       }
-      float mx = s[0];
+      float mx;
+      {
+        float m8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < 128; c += 8)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      }
       const float m_cand = mx * p.scale_log2;
       const bool grow = m_cand > m_run + ATC_RESCALE_LOG2 || (m_run == -INFINITY && m_cand > -INFINITY);
       float alpha = 1.f;
       if (grow) {
-        alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_cand);
+        alpha = (m_run == -INFINITY) ? 0.f : ptx::ex2_approx(m_run - m_cand);
         m_run = m_cand;
         l_run *= alpha;
       }
@@ -293,21 +287,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         ptx::tmem_st_wait();
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float lsum = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 128; c += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = exp2f(fmaf(s[c + 2 * i], p.scale_log2, -m_use));
-          const float p1 = exp2f(fmaf(s[c + 2 * i + 1], p.scale_log2, -m_use));
-          lsum += p0 + p1;
+          const float p0 = ptx::ex2_approx(fmaf(s[c + 2 * i], p.scale_log2, -m_use));
+          const float p1 = ptx::ex2_approx(fmaf(s[c + 2 * i + 1], p.scale_log2, -m_use));
+          ls[i & 3] += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
         }
         ptx::tmem_st16(s_addr + (uint32_t)(c / 2), pk);
       }
       ptx::tmem_st_wait();
-      l_run += lsum;
+      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&pready[tile]);

@@ -16,6 +16,7 @@
 #include "topk.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "compact.cuh"
 
 using namespace quoka;
 
@@ -276,10 +277,21 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
   return QUOKA_OK;
 }
 
+// Rows per (sequence, KV head) block of the compacted cache.
+long long kc_block_rows(const Dims& d, int b_max) {
+  return (long long)align_up((size_t)b_max + d.C, 128);
+}
+
+size_t attn_ws_bytes(const Dims& d, int b_max) {
+  if (d.dt != QUOKA_BF16) return 0;
+  const size_t rows = (size_t)d.batch * d.h_kv * (size_t)kc_block_rows(d, b_max);
+  return 2 * align_up(rows * d.D * 2, 256);
+}
+
 template <int D>
 quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                             const void* k, const void* v, const int32_t* idx, int b_max,
-                            void* out, cudaStream_t st) {
+                            void* out, unsigned char* ws, cudaStream_t st) {
   AttnTcParams p;
   p.h_q = d.h_q;
   p.h_kv = d.h_kv;
@@ -287,18 +299,30 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
   p.C = d.C;
   p.TP = 128 / d.G;
   p.b_max = b_max;
+  p.kc_stride = kc_block_rows(d, b_max);
   p.rows_per_head = rows;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  const size_t kc_rows = (size_t)d.batch * d.h_kv * p.kc_stride;
+  unsigned char* kc = ws;
+  unsigned char* vc = ws + attn_ws_bytes(d, b_max) / 2;
+  cudaError_t e;
+  // 1. the compacted cache: selected rows then the chunk rows, per (sequence, KV head)
+  const long long vecs = (long long)kc_rows * (D * 2 / 16);
+  const int cgrid = (int)std::min<long long>((vecs + CPT_THREADS - 1) / CPT_THREADS, (long long)sm_count() * 16);
+  compact_kv_kernel<D><<<cgrid, CPT_THREADS, 0, st>>>(
+      reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), rows, tab, d.h_kv, d.C,
+      b_max, p.kc_stride, idx, reinterpret_cast<uint4*>(kc), reinterpret_cast<uint4*>(vc), vecs);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "compact launch");
+  // 2. dense attention over it
   CUtensorMap qmap, kmap, vmap;
   quoka_status s;
   if ((s = make_map_bf16(&qmap, q, (uint64_t)d.batch * d.h_q * d.C, D, 64, 1, "q_chunk")) != QUOKA_OK) return s;
-  if ((s = make_map_bf16(&kmap, k, (uint64_t)d.h_kv * rows, D, 64, 1, "k_cache")) != QUOKA_OK) return s;
-  if ((s = make_map_bf16(&vmap, v, (uint64_t)d.h_kv * rows, D, 64, 1, "v_cache")) != QUOKA_OK) return s;
-  cudaError_t e;
+  if ((s = make_map_bf16(&kmap, kc, kc_rows, D, 64, 128, "compacted K")) != QUOKA_OK) return s;
+  if ((s = make_map_bf16(&vmap, vc, kc_rows, D, 64, 128, "compacted V")) != QUOKA_OK) return s;
   const int smem = AtcCfg<D>::SMEM;
   if ((e = ensure_smem(attn_tc_kernel<D>, smem)) != cudaSuccess) return cuda_fail(e, "attn_tc smem");
   dim3 grid((d.C + 2 * p.TP - 1) / (2 * p.TP), d.h_kv, d.batch);
-  attn_tc_kernel<D><<<grid, ATC_THREADS, smem, st>>>(qmap, kmap, vmap, tab, p, idx,
+  attn_tc_kernel<D><<<grid, ATC_THREADS, smem, st>>>(qmap, kmap, vmap, tab, p,
                                                       reinterpret_cast<__nv_bfloat16*>(out));
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_tc launch");
   return QUOKA_OK;
@@ -307,8 +331,8 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
 template <typename T, int D>
 quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                          const void* k, const void* v, const int32_t* idx, int b_max, void* out,
-                         cudaStream_t st) {
-  if (d.dt == QUOKA_BF16) return launch_attn_tc<D>(d, tab, rows, q, k, v, idx, b_max, out, st);
+                         unsigned char* ws, cudaStream_t st) {
+  if (d.dt == QUOKA_BF16) return launch_attn_tc<D>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
   cudaError_t e;
   const int s = attn_simt_smem_bytes<D>();
   if ((e = ensure_smem(attn_simt_kernel<T, D>, s)) != cudaSuccess) return cuda_fail(e, "attn smem");
@@ -378,10 +402,17 @@ quoka_status quoka_select(const quoka_shape* shape, const void* q_chunk, const v
                    : launch_select<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, nq, b_max, idx_out, kept_out, ws, w, st);
 }
 
+size_t sparse_chunk_attn_workspace_size(const quoka_shape* shape, int b_max) {
+  Dims d;
+  if (check_shape(shape, &d) != QUOKA_OK || b_max < 1) return 0;
+  return attn_ws_bytes(d, b_max);
+}
+
 quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk, const void* k_cache,
                                const void* v_cache, const int64_t* kv_off,
                                const int32_t* prefix_len, const int32_t* budget,
-                               const int32_t* idx, int b_max, void* out, void* stream) {
+                               const int32_t* idx, int b_max, void* out, void* workspace,
+                               size_t ws_bytes, void* stream) {
   Dims d;
   quoka_status s = check_shape(shape, &d);
   if (s != QUOKA_OK) return s;
@@ -395,13 +426,20 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk, co
   SeqTable tab;
   long long rows = 0;
   if ((s = build_table(d, kv_off, prefix_len, budget, b_max, &tab, &rows)) != QUOKA_OK) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (d.dt == QUOKA_F32) {
-    return d.D == 64 ? launch_attn<float, 64>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, st)
-                     : launch_attn<float, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, st);
+  const size_t need = attn_ws_bytes(d, b_max);
+  if (need > 0) {
+    if (!workspace) return fail(QUOKA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+    if (!aligned(workspace, 256)) return fail(QUOKA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (ws_bytes < need) return fail(QUOKA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
   }
-  return d.D == 64 ? launch_attn<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, st)
-                   : launch_attn<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, st);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+  if (d.dt == QUOKA_F32) {
+    return d.D == 64 ? launch_attn<float, 64>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st)
+                     : launch_attn<float, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st);
+  }
+  return d.D == 64 ? launch_attn<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st)
+                   : launch_attn<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st);
 }
 
 }  // extern "C"

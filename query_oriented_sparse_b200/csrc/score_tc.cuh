@@ -262,26 +262,34 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         if (!ok) break;
         ptx::tc_fence_after();
         const int nc = min(STC_SLICE, ncols - sl * STC_SLICE);
-        for (int c0 = 0; c0 < nc; c0 += 16) {
-          uint32_t r[16];
-          ptx::tmem_ld16(lane_base + (uint32_t)(buf * STC_SLICE + c0), r);
+        for (int c0 = 0; c0 < nc; c0 += 64) {
+          // up to four 16-column TMEM loads in flight, one wait
+          uint32_t r[4][16];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            if (c0 + q4 * 16 < nc)
+              ptx::tmem_ld16(lane_base + (uint32_t)(buf * STC_SLICE + c0 + q4 * 16), r[q4]);
           ptx::tmem_ld_wait();
-          const int col = sl * STC_SLICE + c0;
-          if (col != 0 && col % p.nkp == 0) {       // a new query head starts here
-            sum += run;
-            run = -INFINITY;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            if (c0 + q4 * 16 >= nc) break;
+            const int col = sl * STC_SLICE + c0 + q4 * 16;
+            if (col != 0 && col % p.nkp == 0) {     // a new query head starts here
+              sum += run;
+              run = -INFINITY;
+            }
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 pr = cp[col + i];
+              v[i] = fmaf(__uint_as_float(r[q4][i]), pr.x, pr.y);
+            }
+#pragma unroll
+            for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+              for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
+            run = fmaxf(run, v[0]);
           }
-          float v[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 pr = cp[col + i];
-            v[i] = fmaf(__uint_as_float(r[i]), pr.x, pr.y);
-          }
-#pragma unroll
-          for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-            for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
-          run = fmaxf(run, v[0]);
         }
         ptx::tc_fence_before();
         __syncwarp();

@@ -38,6 +38,16 @@ def test_library_loads_and_exports_every_declared_symbol():
     assert Bd.version() == 100
 
 
+def test_attn_workspace_size():
+    s = Bd.make_shape(1, 32, 8, 128, 4096, torch.bfloat16)
+    # compacted K and V: 8 heads x (16384 selected + 4096 chunk rows) x 256 B each
+    assert Bd.attn_workspace_size(s, 16384) == 2 * 8 * (16384 + 4096) * 256
+    # blocks are padded to a multiple of 128 rows
+    assert Bd.attn_workspace_size(Bd.make_shape(1, 8, 4, 128, 96, torch.bfloat16), 200) == \
+        2 * 4 * 384 * 256
+    assert Bd.attn_workspace_size(Bd.make_shape(1, 4, 1, 64, 128, torch.float32), 128) == 0
+
+
 def test_workspace_size_is_host_only():
     s = Bd.make_shape(1, 32, 8, 128, 4096, torch.bfloat16)
     n = Bd.select_workspace_size(s, 131072, 128)
@@ -62,10 +72,11 @@ def _select(shape, q=FAKE, k=FAKE, kv_off=(0, 1024), prefix=(512,), nq=8, budget
 
 
 def _attn(shape, q=FAKE, k=FAKE, v=FAKE, kv_off=(0, 1024), prefix=(512,), budget=(64,),
-          idx=FAKE, b_max=64, out=FAKE + 4096):
+          idx=FAKE, b_max=64, out=FAKE + 4096, ws=FAKE, ws_bytes=1 << 30):
     lib = Bd.lib()
     return lib.sparse_chunk_attn(ctypes.byref(shape), q, k, v, Bd._host_i64(kv_off),
-                                 Bd._host_i32(prefix), Bd._host_i32(budget), idx, b_max, out, None)
+                                 Bd._host_i32(prefix), Bd._host_i32(budget), idx, b_max, out, ws,
+                                 ws_bytes, None)
 
 
 @no_gpu
@@ -104,6 +115,9 @@ def test_select_rejects(case, status):
     (dict(k=FAKE + 8), Bd.QUOKA_ERR_INVALID_ARG),
     (dict(budget=(-1,)), Bd.QUOKA_ERR_INVALID_ARG),
     (dict(kv_off=(0, 600)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(ws=None), Bd.QUOKA_ERR_WORKSPACE),
+    (dict(ws_bytes=1000), Bd.QUOKA_ERR_WORKSPACE),
+    (dict(ws=FAKE + 64), Bd.QUOKA_ERR_INVALID_ARG),
 ])
 def test_attn_rejects(case, status):
     shp = dict(batch=1, h_q=8, h_kv=2, head_dim=128, chunk=256, dtype=Bd.QUOKA_BF16)
