@@ -115,9 +115,10 @@ WsLayout ws_layout(const Dims& d, int max_prefix, int nq) {
   WsLayout w;
   w.nk = nq < d.C ? nq : d.C;
   w.nkp = (w.nk + 15) / 16 * 16;
-  w.tc = d.dt == QUOKA_BF16 && w.nkp <= STC_MAXCOLS;
+  w.tc = d.dt == QUOKA_BF16 && w.nkp <= STC_SLICE;
   if (w.tc) {
-    const int hmax = STC_MAXCOLS / w.nkp;
+    // a column group is at most two head-aligned slices of <= 256 columns
+    const int hmax = 2 * (STC_SLICE / w.nkp);
     w.ncg = (d.G + hmax - 1) / hmax;
     w.heads_per_cg = (d.G + w.ncg - 1) / w.ncg;
   } else {
@@ -210,6 +211,7 @@ quoka_status launch_score_tc(const Dims& d, const SeqTable& tab, long long rows,
   p.nkp = w.nkp;
   p.ncg = w.ncg;
   p.heads_per_cg = w.heads_per_cg;
+  p.padded = w.nk < w.nkp ? 1 : 0;
   p.rows_per_head = rows;
   p.pooled_stride = w.pooled_stride;
   p.cg_stride = w.cg_stride;
@@ -250,10 +252,8 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
   float* pooled = reinterpret_cast<float*>(ws + w.pooled);
   cudaError_t e;
 
-  const int s1 = qsub_smem_bytes<D>(d.C);
-  if ((e = ensure_smem(qsub_kernel<T, D>, s1)) != cudaSuccess) return cuda_fail(e, "qsub smem");
-  qsub_kernel<T, D><<<d.batch * d.h_q, QSUB_THREADS, s1, st>>>(
-      reinterpret_cast<const T*>(q), d.h_q, d.C, w.nk, w.nkp, nq, kept_out, qsel, qinv, qbias);
+  qsub_kernel<T, D><<<d.batch * d.h_q * QSUB_CS, QSUB_THREADS, 0, st>>>(
+      reinterpret_cast<const T*>(q), d.C, w.nk, w.nkp, nq, kept_out, qsel, qinv, qbias);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "qsub launch");
 
   if (tab.max_prefix > 0) {
@@ -271,7 +271,10 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
     }
   }
 
-  topk_kernel<<<d.batch * d.h_kv * TOPK_CS, TOPK_THREADS, 0, st>>>(
+  const int tk_keys = std::min((tab.max_prefix + TOPK_CS - 1) / TOPK_CS, TOPK_STAGE_KEYS);
+  const int tk_smem = tk_keys * 4;
+  if ((e = ensure_smem(topk_kernel, tk_smem)) != cudaSuccess) return cuda_fail(e, "topk smem");
+  topk_kernel<<<d.batch * d.h_kv * TOPK_CS, TOPK_THREADS, tk_smem, st>>>(
       pooled, w.pooled_stride, w.ncg, w.cg_stride, 1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
   return QUOKA_OK;

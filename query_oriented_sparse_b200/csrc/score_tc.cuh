@@ -10,11 +10,15 @@
 // traffic is one read of the prefix keys.
 //
 // Persistent CTAs each take a contiguous run of work units (sequence, KV head, column
-// group, 128-key tile).  A column group is up to 512 kept-query columns (whole heads);
-// its operand block stays resident in shared memory while key tiles stream through a
-// ring of 16 KB K-block stages loaded by TMA (128-byte swizzle).  Warp 0 issues TMA,
-// one thread of warp 1 issues the MMAs into two 256-column TMEM slices, warps 2-5
-// drain one slice while the tensor core fills the other.
+// group, 128-key tile).  A column group is up to 2 x 256 kept-query columns (whole
+// heads); its operand block stays resident in shared memory while key tiles stream
+// through a ring of 16 KB K-block stages loaded by TMA (128-byte swizzle).  Warp 0
+// issues TMA, one thread of warp 1 issues the MMAs of each tile as one or two column
+// slices (cut on head boundaries) into two 256-column TMEM accumulators, and two
+// epilogue warpgroups (warps 2-5 and 6-9) drain alternate accumulators, so every SM
+// sub-partition has two warps to interleave.  When a tile has two slices, the group
+// that drains the second one adds the other group's partial sum and |k|^2 share,
+// handed over through a shared-memory slot guarded by an mbarrier pair.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -22,13 +26,14 @@ namespace quoka {
 
 constexpr int STC_BM = 128;        // keys per tile (TMEM lanes)
 constexpr int STC_MAXCOLS = 512;   // kept-query columns per column group
-constexpr int STC_SLICE = 256;     // MMA N per accumulator slice
+constexpr int STC_SLICE = 256;     // max MMA N per accumulator slice
 constexpr int STC_NBUF = 2;        // accumulator slices held in TMEM
-constexpr int STC_THREADS = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int STC_THREADS = 320;   // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9 epilogue
 constexpr int STC_QBOX = 16;       // rows per TMA box of the kept-query block
 
 struct ScoreTcParams {
   int h_kv, G, nkp, ncg, heads_per_cg;
+  int padded;                   // nonzero when heads carry padding columns (bias needed)
   int total_units;
   long long rows_per_head;
   long long pooled_stride;      // floats per (sequence, KV head) row
@@ -45,9 +50,12 @@ struct StcCfg {
   static constexpr int QBLK_BYTES = STC_MAXCOLS * 128; // one K-block of the query block
   static constexpr int Q_BYTES = QBLK_BYTES * KB;
   static constexpr int K_BYTES = STAGE_BYTES * NST;
-  static constexpr int CP_BYTES = STC_MAXCOLS * 8;     // (1/|q|, bias) per column
-  static constexpr int NBAR = 2 * NST + 2 + 2 * STC_NBUF;
-  static constexpr int SMEM = 1024 + Q_BYTES + K_BYTES + CP_BYTES + NBAR * 8 + 16;
+  // 1/|q| and bias per column; twice the columns so the masked tail of a 64-column
+  // batch past a slice end still reads inside the arrays
+  static constexpr int CP_BYTES = 2 * STC_MAXCOLS * 8;
+  static constexpr int NBAR = 2 * NST + 2 + 2 * STC_NBUF + 4;
+  static constexpr int MERGE_BYTES = 2 * STC_BM * 8;   // two (partial sum, |k|^2 share) slots
+  static constexpr int SMEM = 1024 + Q_BYTES + K_BYTES + CP_BYTES + MERGE_BYTES + NBAR * 8 + 16;
 };
 
 __device__ __forceinline__ void stc_decode(const ScoreTcParams& p, const SeqTable& tab, int u,
@@ -78,14 +86,18 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + Cfg::Q_BYTES;
-  float2* cp = reinterpret_cast<float2*>(sK + Cfg::K_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(cp) + Cfg::CP_BYTES);
+  float* cpi = reinterpret_cast<float*>(sK + Cfg::K_BYTES);     // 1/|q| per column
+  float* cpb = cpi + 2 * STC_MAXCOLS;                             // bias per column
+  float* merge = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(cpi) + Cfg::CP_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(merge) + Cfg::MERGE_BYTES);
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + NST;
   uint64_t* qfull = bars + 2 * NST;
   uint64_t* qempty = qfull + 1;
   uint64_t* accfull = qfull + 2;
   uint64_t* accempty = accfull + STC_NBUF;
+  uint64_t* mfull = accempty + STC_NBUF;   // [2] partial sum of slice 0 written
+  uint64_t* mempty = mfull + 2;            // [2] slot consumed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -96,13 +108,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       ptx::mbar_init(&kfull[s], 1);
-      ptx::mbar_init(&kempty[s], 1 + 4);
+      ptx::mbar_init(&kempty[s], 1 + 8);
     }
     ptx::mbar_init(qfull, 1);
     ptx::mbar_init(qempty, 1);
     for (int s = 0; s < STC_NBUF; ++s) {
       ptx::mbar_init(&accfull[s], 1);
       ptx::mbar_init(&accempty[s], 4);
+      ptx::mbar_init(&mfull[s], 128);
+      ptx::mbar_init(&mempty[s], 128);
     }
     ptx::fence_mbar_init();
   }
@@ -180,19 +194,22 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         }
         if (!ok) break;
         ptx::tc_fence_after();
-        for (int sl = 0; sl * STC_SLICE < ncols && ok; ++sl, ++nsl_done) {
+        const int nsl = ncols > STC_SLICE ? 2 : 1;
+        const int cols0 = nsl == 2 ? ((ncols / p.nkp + 1) / 2) * p.nkp : ncols;
+        for (int sl = 0; sl < nsl && ok; ++sl, ++nsl_done) {
           const int buf = nsl_done & 1;
           const uint32_t bph = (uint32_t)(nsl_done >> 1) & 1u;
           ok = ptx::mbar_wait(&accempty[buf], bph ^ 1u);
           if (!ok) break;
           ptx::tc_fence_after();
-          const int nc = min(STC_SLICE, ncols - sl * STC_SLICE);
+          const int c0 = sl == 0 ? 0 : cols0;
+          const int nc = sl == 0 ? cols0 : ncols - cols0;
           const uint32_t idesc = ptx::idesc_bf16(128, nc, false);
           const uint32_t d_tmem = tmem + (uint32_t)(buf * STC_SLICE);
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
             const uint32_t a0 = ptx::smem_u32(sK + st[kb] * Cfg::STAGE_BYTES);
-            const uint32_t b0 = ptx::smem_u32(sQ + kb * Cfg::QBLK_BYTES + sl * STC_SLICE * 128);
+            const uint32_t b0 = ptx::smem_u32(sQ + kb * Cfg::QBLK_BYTES + c0 * 128);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               ptx::mma_bf16_ss(d_tmem, ptx::sdesc_sw128(a0 + ks * 32, 16, 1024),
@@ -206,11 +223,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       }
     }
   } else {
-    // ---------------- epilogue: warps 2..5, one key per thread ----------------
+    // ---------------- epilogue: two groups (warps 2-5, 6-9), one key per thread ----------
+    const int set = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    int stage = 0, cur = -1, nsl_done = 0, ncols = 0;
+    int stage = 0, cur = -1, nsl_done = 0, ncols = 0, nmerge = 0;
     uint32_t kph = 0;
     bool ok = true;
     for (int u = u_lo; u < u_hi && ok; ++u) {
@@ -218,22 +236,41 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       stc_decode(p, tab, u, b, g, cg, tile);
       const int key3 = (b * p.h_kv + g) * p.ncg + cg;
       if (key3 != cur) {
-        ptx::named_bar(1, 128);
+        ptx::named_bar(1, 256);
         const int h0 = cg * p.heads_per_cg;
         ncols = (min(p.G, h0 + p.heads_per_cg) - h0) * p.nkp;
         const size_t c0 = (size_t)(b * p.h_kv + g) * p.G * p.nkp + (size_t)h0 * p.nkp;
-        for (int c = threadIdx.x - 64; c < ncols; c += 128) cp[c] = make_float2(qinv[c0 + c], qbias[c0 + c]);
-        ptx::named_bar(1, 128);
+        for (int c = threadIdx.x - 64; c < ncols; c += 256) {
+          cpi[c] = qinv[c0 + c];
+          cpb[c] = qbias[c0 + c];
+        }
+        ptx::named_bar(1, 256);
         cur = key3;
       }
-      // |k| of this thread's key from the swizzled tile in shared memory
-      float ss = 0.f;
+      const int nsl = ncols > STC_SLICE ? 2 : 1;
+      const int cols0 = nsl == 2 ? ((ncols / p.nkp + 1) / 2) * p.nkp : ncols;
+      const int fin = (nsl_done + nsl - 1) & 1;   // group draining the tile's last slice
       int st[KB];
+      uint32_t sph[KB];                            // ring slot and its phase per K-block
       for (int kb = 0; kb < KB; ++kb) {
         st[kb] = stage;
-        if (ok) ok = ptx::mbar_wait(&kfull[stage], kph);
+        sph[kb] = kph;
+        if (++stage == NST) { stage = 0; kph ^= 1u; }
+      }
+      // |k|^2 of this thread's key from the swizzled tile in shared memory: the owner of
+      // a one-slice tile reads every K-block, a two-slice tile splits them
+      int kb_lo = 0, kb_hi = 0;
+      if (nsl == 1) {
+        if (set == fin) kb_hi = KB;
+      } else {
+        kb_lo = (set == fin) ? KB / 2 : 0;
+        kb_hi = (set == fin) ? KB : KB / 2;
+      }
+      float ss = 0.f;
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+        if (ok) ok = ptx::mbar_wait(&kfull[st[kb]], sph[kb]);
         if (ok) {
-          const uint8_t* rp = sK + stage * Cfg::STAGE_BYTES + row * 128;
+          const uint8_t* rp = sK + st[kb] * Cfg::STAGE_BYTES + row * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 v = *reinterpret_cast<const uint4*>(rp + ((c ^ (row & 7)) << 4));
@@ -246,57 +283,104 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
             }
           }
         }
-        if (++stage == NST) { stage = 0; kph ^= 1u; }
       }
       ok = __all_sync(0xffffffffu, ok);
       if (lane == 0)
         for (int kb = 0; kb < KB; ++kb) ptx::mbar_arrive(&kempty[st[kb]]);
       if (!ok) break;
-      const float knorm = sqrtf(ss);
 
-      float run = -INFINITY, sum = 0.f;
-      for (int sl = 0; sl * STC_SLICE < ncols && ok; ++sl, ++nsl_done) {
+      float sum = 0.f;
+      for (int sl = 0; sl < nsl && ok; ++sl, ++nsl_done) {
         const int buf = nsl_done & 1;
+        if (buf != set) continue;
         const uint32_t bph = (uint32_t)(nsl_done >> 1) & 1u;
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&accfull[buf], bph));
         if (!ok) break;
         ptx::tc_fence_after();
-        const int nc = min(STC_SLICE, ncols - sl * STC_SLICE);
+        const int cbase = sl == 0 ? 0 : cols0;
+        const int nc = sl == 0 ? cols0 : ncols - cols0;
+        float run = -INFINITY;
+        int to_boundary = p.nkp;                 // columns left in the current head
         for (int c0 = 0; c0 < nc; c0 += 64) {
-          // up to four 16-column TMEM loads in flight, one wait
-          uint32_t r[4][16];
+          // up to 64 columns of TMEM loads in flight per wait
+          uint32_t r[2][32];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            if (c0 + q4 * 16 < nc)
-              ptx::tmem_ld16(lane_base + (uint32_t)(buf * STC_SLICE + c0 + q4 * 16), r[q4]);
+          for (int q4 = 0; q4 < 2; ++q4)
+            if (c0 + q4 * 32 < nc)
+              ptx::tmem_ld32(lane_base + (uint32_t)(buf * STC_SLICE + c0 + q4 * 32), r[q4]);
           ptx::tmem_ld_wait();
+          // four independent 16-column maxima of (s * 1/|q| + bias); groups past the
+          // slice end are -inf.  Columns of a group always belong to one query head.
+          float gm[4];
+          const float4* ci4 = reinterpret_cast<const float4*>(cpi + cbase + c0);
+          const float4* cb4 = reinterpret_cast<const float4*>(cpb + cbase + c0);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            if (c0 + q4 * 16 >= nc) break;
-            const int col = sl * STC_SLICE + c0 + q4 * 16;
-            if (col != 0 && col % p.nkp == 0) {     // a new query head starts here
-              sum += run;
-              run = -INFINITY;
-            }
+          for (int q8 = 0; q8 < 4; ++q8) {
             float v[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float2 pr = cp[col + i];
-              v[i] = fmaf(__uint_as_float(r[q4][i]), pr.x, pr.y);
+            for (int i = 0; i < 4; ++i) {
+              const float4 sc = ci4[q8 * 4 + i];
+              const uint32_t* rr = &r[q8 >> 1][(q8 & 1) * 16 + 4 * i];
+              const float2 s01 = make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1]));
+              const float2 s23 = make_float2(__uint_as_float(rr[2]), __uint_as_float(rr[3]));
+              float2 v01, v23;
+              if (p.padded) {
+                const float4 bi = cb4[q8 * 4 + i];
+                v01 = ptx::fma2(s01, make_float2(sc.x, sc.y), make_float2(bi.x, bi.y));
+                v23 = ptx::fma2(s23, make_float2(sc.z, sc.w), make_float2(bi.z, bi.w));
+              } else {
+                v01 = ptx::mul2(s01, make_float2(sc.x, sc.y));
+                v23 = ptx::mul2(s23, make_float2(sc.z, sc.w));
+              }
+              v[4 * i] = v01.x; v[4 * i + 1] = v01.y; v[4 * i + 2] = v23.x; v[4 * i + 3] = v23.y;
             }
+            const float a0 = ptx::max3(v[0], v[1], v[2]), a1 = ptx::max3(v[3], v[4], v[5]);
+            const float a2 = ptx::max3(v[6], v[7], v[8]), a3 = ptx::max3(v[9], v[10], v[11]);
+            const float a4 = ptx::max3(v[12], v[13], v[14]);
+            const float m = fmaxf(ptx::max3(a0, a1, a2), ptx::max3(a3, a4, v[15]));
+            gm[q8] = (c0 + q8 * 16 < nc) ? m : -INFINITY;
+          }
+          const int ng = min(4, (nc - c0) >> 4);
 #pragma unroll
-            for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-              for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
-            run = fmaxf(run, v[0]);
+          for (int q8 = 0; q8 < 4; ++q8) {
+            if (q8 < ng) {
+              if (to_boundary == 0) {              // a new query head starts here
+                sum += run;
+                run = -INFINITY;
+                to_boundary = p.nkp;
+              }
+              to_boundary -= 16;
+              run = fmaxf(run, gm[q8]);
+            }
           }
         }
+        sum += run;
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&accempty[buf]);
       }
       if (!ok) break;
-      sum += run;
+      if (nsl == 2) {
+        const int slot = nmerge & 1;
+        const uint32_t mph = (uint32_t)(nmerge >> 1) & 1u;
+        ++nmerge;
+        if (set != fin) {                           // hand slice 0's partial sum over
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(&mempty[slot], mph ^ 1u));
+          if (!ok) break;
+          reinterpret_cast<float2*>(merge)[slot * STC_BM + row] = make_float2(sum, ss);
+          ptx::mbar_arrive(&mfull[slot]);
+          continue;
+        }
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&mfull[slot], mph));
+        if (!ok) break;
+        const float2 other = reinterpret_cast<float2*>(merge)[slot * STC_BM + row];
+        sum = other.x + sum;
+        ss = other.y + ss;
+        ptx::mbar_arrive(&mempty[slot]);
+      } else if (set != fin) {
+        continue;
+      }
+      const float knorm = sqrtf(ss);
       const int j = tile * STC_BM + row;
       if (j < tab.prefix[b]) {
         const float s = knorm > 0.f ? (p.ncg == 1 ? sum * p.inv_G : sum) / knorm : 0.f;

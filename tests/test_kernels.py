@@ -34,6 +34,11 @@ CASES = [
       recipe="rank4", seed=13),
     C("long_tail_bf16", h_q=8, h_kv=1, head_dim=128, chunk=300, prefix=5000, nq=40, budget=613,
       recipe="heavy", seed=14),
+    # 3 heads of 112 padded rows per column group: two uneven head-aligned slices
+    C("uneven_slices", h_q=12, h_kv=2, head_dim=128, chunk=150, prefix=3000, nq=100, budget=300,
+      recipe="rank4", seed=17),
+    # kept queries wider than one accumulator slice per head: CUDA-core scoring
+    C("wide_nq", h_q=4, h_kv=2, head_dim=64, chunk=400, prefix=900, nq=300, budget=200, seed=18),
 ]
 
 
