@@ -12,10 +12,15 @@
 // TMA loads per operand (128-byte swizzle) into a 3-stage K ring and a 2-stage V ring.
 //
 // TMEM holds S0, S1 (128 x 128 fp32 logits of each tile) and O0, O1 (128 x d fp32).
-// Warp 0 loads, one thread of warp 1 issues tcgen05.mma, warps 2-5 and 6-9 run the
-// softmax of tile 0 and tile 1 (one thread per query row) so that one tile's
-// exponentials overlap the other tile's MMAs.  P is written back as bf16 over the
-// first 64 columns of S and consumed from TMEM by the P.V MMA (A operand in TMEM).
+// Warp 0 loads, one thread of warp 1 issues tcgen05.mma, warps 2-9 and 10-17 run the
+// softmax of tile 0 and tile 1, so one tile's softmax overlaps the other tile's MMAs.
+// Each query row is shared by two warps of the same SM sub-partition, one per 64-key
+// half of the block (one thread per row and half): the exponentials of a tile run on
+// 8 warps, two per sub-partition, which is what it takes to keep the multi-function
+// units busy.  The two halves of a row agree on the block maximum through shared memory
+// under a 64-thread named barrier.  P is written back as bf16 into TMEM inside each
+// half's own S columns (keys 0-63 -> columns 0-31, keys 64-127 -> columns 96-127) and
+// consumed from TMEM by the P.V MMA (A operand in TMEM).
 // The online softmax keeps its running max per row in fp32 and rescales O in TMEM
 // only when the max grows by more than 2^8, so the exponent stays bounded.
 #pragma once
@@ -23,7 +28,7 @@
 
 namespace quoka {
 
-constexpr int ATC_THREADS = 320;   // warp 0 load, warp 1 MMA, 2-5 softmax tile 0, 6-9 tile 1
+constexpr int ATC_THREADS = 576;   // warp 0 load, warp 1 MMA, 2-9 softmax tile 0, 10-17 tile 1
 constexpr int ATC_KST = 3;         // K stages
 constexpr int ATC_VST = 2;         // V stages
 constexpr float ATC_RESCALE_LOG2 = 8.0f;
@@ -42,8 +47,10 @@ struct AtcCfg {
   static constexpr int Q_BYTES = 2 * TILE_BYTES;
   static constexpr int K_BYTES = ATC_KST * TILE_BYTES;
   static constexpr int V_BYTES = ATC_VST * TILE_BYTES;
+  // qfull, K and V full/empty rings, and per tile sfull, pready, odone
   static constexpr int NBAR = 1 + 2 * ATC_KST + 2 * ATC_VST + 2 + 2 + 2;
-  static constexpr int SMEM = 1024 + Q_BYTES + K_BYTES + V_BYTES + NBAR * 8 + 16;
+  static constexpr int XBUF = 2 * 128 * 4;         // per-row exchange slots of both tiles
+  static constexpr int SMEM = 1024 + Q_BYTES + K_BYTES + V_BYTES + NBAR * 8 + 16 + XBUF;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -74,6 +81,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   uint64_t* pready = sfull + 2;         // [2]
   uint64_t* odone = pready + 2;         // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(odone + 2);
+  float* xbuf = reinterpret_cast<float*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.z, g = blockIdx.y;
@@ -92,7 +100,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     for (int s = 0; s < ATC_VST; ++s) { ptx::mbar_init(&vfull[s], 1); ptx::mbar_init(&vempty[s], 1); }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sfull[i], 1);
-      ptx::mbar_init(&pready[i], 4);
+      ptx::mbar_init(&pready[i], 8);
       ptx::mbar_init(&odone[i], 1);
     }
     ptx::fence_mbar_init();
@@ -158,28 +166,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const uint32_t idesc_s = ptx::idesc_bf16(128, 128, false);
       const uint32_t idesc_o = ptx::idesc_bf16(128, D, true);
       bool ok = ptx::mbar_wait(qfull, 0);
+      // Descriptor halves: only the start-address field (low half, address >> 4) moves as
+      // the MMAs step through k, the tile and the ring stage.
+      const uint64_t q_d = ptx::sdesc_sw128(ptx::smem_u32(sQ), 16, 1024);
+      const uint64_t k_d = ptx::sdesc_sw128(ptx::smem_u32(sK), 16, 1024);
+      const uint64_t v_d = ptx::sdesc_sw128(ptx::smem_u32(sV), 16384, 1024);
+      const uint32_t q_lo = (uint32_t)q_d, q_hi = (uint32_t)(q_d >> 32);
+      const uint32_t k_lo = (uint32_t)k_d, k_hi = (uint32_t)(k_d >> 32);
+      const uint32_t v_lo = (uint32_t)v_d, v_hi = (uint32_t)(v_d >> 32);
+      constexpr uint32_t TILE16 = (uint32_t)Cfg::TILE_BYTES >> 4;
       auto issue_s = [&](int i, int j) {
-        const int ks = j % ATC_KST;
-        const uint32_t a0 = ptx::smem_u32(sQ + i * Cfg::TILE_BYTES);
-        const uint32_t b0 = ptx::smem_u32(sK + ks * Cfg::TILE_BYTES);
+        const uint32_t a0 = q_lo + (uint32_t)i * TILE16;
+        const uint32_t b0 = k_lo + (uint32_t)(j % ATC_KST) * TILE16;
+        const uint32_t d = tmem + (uint32_t)(i * 128);
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            ptx::mma_bf16_ss(tmem + (uint32_t)(i * 128),
-                             ptx::sdesc_sw128(a0 + kb * 16384 + k * 32, 16, 1024),
-                             ptx::sdesc_sw128(b0 + kb * 16384 + k * 32, 16, 1024), idesc_s,
-                             (kb | k) ? 1u : 0u);
+            ptx::mma_bf16_ss_lh(d, a0 + (uint32_t)(kb * 1024 + k * 2), q_hi, b0 + (uint32_t)(kb * 1024 + k * 2),
+                                k_hi, idesc_s, (kb | k) ? 1u : 0u);
         ptx::tc_commit(&sfull[i]);
       };
       auto issue_pv = [&](int i, int j) {
-        const int vs = j % ATC_VST;
-        const uint32_t b0 = ptx::smem_u32(sV + vs * Cfg::TILE_BYTES);
+        const uint32_t b0 = v_lo + (uint32_t)(j % ATC_VST) * TILE16;
+        const uint32_t d = tmem + (uint32_t)(256 + i * 128), pa = tmem + (uint32_t)(i * 128);
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int k = 0; k < 8; ++k)                          // 16 keys per MMA
-          ptx::mma_bf16_ts(tmem + (uint32_t)(256 + i * 128), tmem + (uint32_t)(i * 128 + k * 8),
-                           ptx::sdesc_sw128(b0 + k * 2048, 16384, 1024), idesc_o,
-                           (j > 0 || k > 0) ? 1u : 0u);
+          ptx::mma_bf16_ts_lh(d, pa + (uint32_t)(k < 4 ? k * 8 : 96 + (k - 4) * 8), b0 + (uint32_t)(k * 128),
+                              v_hi, idesc_o, k > 0 ? 1u : acc0);
         ptx::tc_commit(&odone[i]);
       };
       if (ok) ok = ptx::mbar_wait(&kfull[0], 0);
@@ -215,36 +230,63 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       }
     }
   } else {
-    // ---------------- softmax: warps 2-5 tile 0, warps 6-9 tile 1 ----------------
-    const int tile = (warp - 2) >> 2;
+    // ---------------- softmax: warps 2-9 tile 0, warps 10-17 tile 1 ----------------
+    // Warp w serves TMEM lanes 32 * (w % 4) .. + 31 (one query row per thread) and key
+    // half (w - 2) / 4 % 2 of every block; the two warps of a row exchange block maxima
+    // (and at the end row sums) through shared memory under a 64-thread named barrier.
+    const int tile = (warp - 2) >> 3;
+    const int half = ((warp - 2) >> 2) & 1;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                      // row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + (uint32_t)(tile * 128);
-    const uint32_t o_addr = tmem + lane_off + (uint32_t)(256 + tile * 128);
+    const uint32_t s_addr = tmem + lane_off + (uint32_t)(tile * 128 + half * 64);
+    const uint32_t p_addr = tmem + lane_off + (uint32_t)(tile * 128 + half * 96);
+    constexpr int DH = D / 2;                               // O columns of this half
+    const uint32_t o_addr = tmem + lane_off + (uint32_t)(256 + tile * 128 + half * DH);
+    float* xslot = xbuf + tile * 128 + r;
+    const int bar_id = 1 + tile * 4 + quarter;
+    // half 0 posts v, half 1 combines it with its own and posts the result for half 0
+    auto exchange = [&](float v, bool is_max) -> float {
+      if (half == 0) *xslot = v;
+      ptx::named_bar(bar_id, 64);
+      float res = v;
+      if (half == 1) {
+        res = is_max ? fmaxf(v, *xslot) : v + *xslot;
+        *xslot = res;
+      }
+      ptx::named_bar(bar_id, 64);
+      if (half == 0) res = *xslot;
+      return res;
+    };
     const int hl = r / p.TP;
     const int t = t0 + tile * p.TP + r % p.TP;
     const bool row_valid = hl < p.G && t < p.C;
     const int tmin = t0 + tile * p.TP;                      // smallest position in this tile
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < nblk && ok; ++j) {
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&sfull[tile], (uint32_t)j & 1u));
-      if (!ok) break;
+    // Both warps of a row pair take part in exactly one exchange per block and one at
+    // the end, whatever happens, so the named barrier can never wait for a warp that left:
+    // after a failed (timed-out) wait a warp skips the work but keeps the exchanges.
+    for (int j = 0; j < nblk; ++j) {
+      if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&sfull[tile], (uint32_t)j & 1u));
+      if (!ok) {
+        (void)exchange(0.f, true);
+        continue;
+      }
       ptx::tc_fence_after();
-      float s[128];
+      float s[64];
 #pragma unroll
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         uint32_t u[32];
         ptx::tmem_ld32(s_addr + (uint32_t)c, u);
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(u[i]);
       }
       ptx::tmem_ld_wait();
-      const int kb0 = j * 128;
-      if (kb0 + 127 >= nsel + tmin || kb0 + 127 >= nkeys) {  // block reaches the causal part
+      const int kb0 = j * 128 + half * 64;
+      if (kb0 + 63 >= nsel + tmin || kb0 + 63 >= nkeys) {   // keys reach the causal part
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
+        for (int c = 0; c < 64; ++c) {
           const int kk = kb0 + c;
           const bool valid = kk < nkeys && (kk < nsel || kk - nsel <= t);
           if (!valid) s[c] = -INFINITY;
@@ -252,15 +294,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       }
       float mx;
       {
-        float m8[8];
+        float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = s[i];
-#pragma unroll
-        for (int c = 8; c < 128; c += 8)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int c = 4; c < 60; c += 8) {
+          m0 = ptx::max3(m0, s[c], s[c + 1]);
+          m1 = ptx::max3(m1, s[c + 2], s[c + 3]);
+          m2 = ptx::max3(m2, s[c + 4], s[c + 5]);
+          m3 = ptx::max3(m3, s[c + 6], s[c + 7]);
+        }
+        m0 = ptx::max3(m0, s[60], s[61]);
+        m1 = ptx::max3(m1, s[62], s[63]);
+        mx = exchange(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), true);
       }
       const float m_cand = mx * p.scale_log2;
       const bool grow = m_cand > m_run + ATC_RESCALE_LOG2 || (m_run == -INFINITY && m_cand > -INFINITY);
@@ -270,26 +314,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         m_run = m_cand;
         l_run *= alpha;
       }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O holds blocks 0..j-1 once the previous P.V of this tile has finished
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&odone[tile], (uint32_t)(j - 1) & 1u));
-        if (!ok) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D; c += 16) {
-          uint32_t u[16];
-          ptx::tmem_ld16(o_addr + (uint32_t)c, u);
-          ptx::tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          ptx::tmem_st16(o_addr + (uint32_t)c, u);
-        }
-        ptx::tmem_st_wait();
-      }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -298,23 +326,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           ls[i & 3] += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
         }
-        ptx::tmem_st16(s_addr + (uint32_t)(c / 2), pk);
+        ptx::tmem_st16(p_addr + (uint32_t)(c / 2), pk);
+      }
+      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      if (ok && j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O holds blocks 0..j-1 once the previous P.V of this tile has finished
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&odone[tile], (uint32_t)(j - 1) & 1u));
+        if (ok) ptx::tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < (ok ? DH : 0); c += 16) {
+          uint32_t u[16];
+          ptx::tmem_ld16(o_addr + (uint32_t)c, u);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          ptx::tmem_st16(o_addr + (uint32_t)c, u);
+        }
       }
       ptx::tmem_st_wait();
-      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&pready[tile]);
+      if (ok && lane == 0) ptx::mbar_arrive(&pready[tile]);
     }
-    // epilogue: O / l -> bf16 rows of out[b, g*G + hl, t, :]
+    // epilogue: O / l -> bf16 rows of out[b, g*G + hl, t, :], this half's columns
     if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&odone[tile], (uint32_t)(nblk - 1) & 1u));
+    const float l_row = exchange(ok ? l_run : 0.f, false);   // every pair member reaches this
     if (ok) {
       ptx::tc_fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
       __nv_bfloat16* orow = out + ((size_t)(b * p.h_q + g * p.G + (row_valid ? hl : 0)) * p.C +
-                                   (row_valid ? t : 0)) * D;
+                                   (row_valid ? t : 0)) * D + half * DH;
 #pragma unroll
-      for (int c = 0; c < D; c += 16) {
+      for (int c = 0; c < DH; c += 16) {
         uint32_t u[16];
         ptx::tmem_ld16(o_addr + (uint32_t)c, u);
         ptx::tmem_ld_wait();
