@@ -36,6 +36,23 @@ METRIC = "chunked-prefill sparse-attn tokens/s (select+attend) and % of roofline
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 LAUNCHES_PER_STEP = 5  # qsub, score, top-k, compaction, attention
+# DRAM traffic of one attention-kernel launch on the 128K-context workload
+# (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture, summarised in
+# profiles/attn_tc_kernel_ctx_128k.md), valid only for the kernel sources it was taken
+# on: the digest below covers them, and a changed kernel reports null.
+ATTN_TRAFFIC = {"workload": "ctx_128k", "bytes": 117.492992e6 + 18.832384e6,
+                "sources": ['query_oriented_sparse_b200/csrc/attn_tc.cuh', 'query_oriented_sparse_b200/csrc/tc_ptx.cuh'], "sha256_16": "74f457a2a89ca874"}
+
+
+def attn_traffic(w):
+    import hashlib
+    if w.name != ATTN_TRAFFIC["workload"]:
+        return None
+    h = hashlib.sha256()
+    for f in ATTN_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return ATTN_TRAFFIC["bytes"] if h.hexdigest()[:16] == ATTN_TRAFFIC["sha256_16"] else None
 
 
 def load_peaks():
@@ -73,38 +90,84 @@ def roofline_us(st, peaks):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons with nvidia-smi while the timed region runs."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the active clock-event (throttle) reasons while the timed
+    region runs: NVML reads from a thread every millisecond (read-only queries), so even
+    a region of a few milliseconds gets samples; nvidia-smi at 200 ms if NVML is absent."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.sel = str(device_index)
+        self.device_index = device_index
+        self.sm, self.reasons, self.max_mhz, self.source = [], set(), None, None
+        self.stop = threading.Event()
+        self.thread = self.proc = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
         try:
-            uuid = torch.cuda.get_device_properties(device_index).uuid
-            self.sel = "GPU-" + str(uuid)
+            uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(
+                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
         except Exception:
-            pass
-        self.proc = None
-        self.lines = []
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
+
+    def _poll(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                mask = int(get_reasons(h))
+                for name, bit in self.REASONS:
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.001)
 
     def __enter__(self):
         try:
+            nv, h = self._nvml_handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.source = "nvml 1 ms"
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", self.sel, "-lms", "200"], stdout=subprocess.PIPE,
+                ["nvidia-smi", f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.device_index), "-lms", "200"], stdout=subprocess.PIPE,
                 stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi 200 ms"
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
         except Exception:
             self.proc = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
+        for ln in self.proc.stdout:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                self.sm.append(float(parts[0]))
+                self.max_mhz = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    self.reasons.add(n)
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             time.sleep(0.25)
             self.proc.terminate()
@@ -112,26 +175,14 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.sm:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.sm), "source": self.source}
 
 
 # --------------------------------------------------------------------------------------
@@ -210,6 +261,17 @@ def run_reference(args, w):
 # --------------------------------------------------------------------------------------
 # GPU arm
 # --------------------------------------------------------------------------------------
+
+def max_over_ranks(vals, device):
+    """Element-wise maximum of per-rank timings over the process group (the slowest
+    rank sets the job's time); the values themselves on a single process."""
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(x) for x in vals]
+    m = torch.tensor([float(x) for x in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(m, op=dist.ReduceOp.MAX)
+    return m.tolist()
+
 
 def run_ours(args, w):
     from query_oriented_sparse_b200 import binding as Bd
@@ -309,12 +371,7 @@ def run_ours(args, w):
     assert torch.equal(out_h.to(dev), out)
 
     tokens = w.batch * C
-    if world > 1:
-        m = torch.tensor([total_s, sum(e2e_ms) / 1e3], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(m, op=torch.distributed.ReduceOp.MAX)
-        total_s, e2e_total_s = m.tolist()
-    else:
-        e2e_total_s = sum(e2e_ms) / 1e3
+    total_s, e2e_total_s = max_over_ranks([total_s, sum(e2e_ms) / 1e3], dev)
     value = world * args.steps * tokens / total_s
     e2e_value = world * args.steps * tokens / e2e_total_s
 
@@ -339,7 +396,8 @@ def run_ours(args, w):
                      "attn": statistics.mean(att_ms) * 1e3},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                     "traffic": None, "kernel": "sparse_chunk_attn",
+                     "traffic": attn_traffic(w),
+                     "kernel": "attn_tc_kernel, timed as the sparse_chunk_attn call (compaction + attention)",
                      "peak_source": f"{peak_src} bf16 dense (burst)"},
         "path_roofline": {"roofline_us": path_roof_us, "stage_roofline_us": rl,
                           "measured_us": total_s * 1e6 / args.steps,

@@ -1,0 +1,84 @@
+"""Host-side logic of bench.py that needs no GPU: the max-over-ranks timing reduction
+on a world_size-2 gloo group, the reference arm's behaviour on ranks other than 0,
+and the algorithmic bytes/FLOPs of the 128K-context step behind the roofline."""
+import io
+import json
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from query_oriented_sparse_b200 import workloads as W  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # each rank times a different step; every rank must see the slowest one
+        got = bench.max_over_ranks([1.0 + rank, 10.0 - rank], torch.device("cpu"))
+        out_q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0] == res[1] == [2.0, 10.0]
+
+
+def test_max_over_ranks_single_process():
+    assert bench.max_over_ranks([3, 4.5], torch.device("cpu")) == [3.0, 4.5]
+
+
+def test_reference_arm_other_ranks_exit_quietly(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    args = type("A", (), {"gpus": 2, "steps": 1, "warmup": 0})()
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        rc = bench.run_reference(args, W.WORKLOADS["gqa_8k"])
+    assert rc == 0 and buf.getvalue() == ""
+
+
+def test_stage_model_ctx_128k():
+    """Algorithmic work of one 128K-context step: scoring 2*H_q*Nq*P*d flops over the
+    whole prefix, attention 4*d*H_q*(C*B + C(C+1)/2) flops over selected + causal keys."""
+    w = W.WORKLOADS["ctx_128k"]
+    st = bench.stage_model(w)
+    P, C, B, d = 131072, 4096, 16384, 128
+    assert st["score"]["flops"] == 2.0 * 32 * 128 * P * d
+    assert st["attn"]["flops"] == 4.0 * d * 32 * (C * B + C * (C + 1) / 2)
+    assert st["score"]["bytes"] == 8 * P * d * 2 + 32 * 128 * d * 2
+    assert st["attn"]["bytes"] == 2 * 32 * C * d * 2 + 2 * 8 * (B + C) * d * 2 + 8 * B * 4
+    rl = bench.roofline_us(st, {"hbm_gbs": 6440.7, "bf16_tflops": 1687.0, "bf16_tflops_sustained": 1436.0})
+    assert abs(rl["attn"] - 733.2) < 0.1 and abs(rl["score"] - 81.5) < 0.1
+    assert abs(sum(rl.values()) - 820.2) < 0.1
+
+
+def test_attn_traffic_is_pinned_to_workload():
+    assert bench.attn_traffic(W.WORKLOADS["gqa_8k"]) is None
+    t = bench.attn_traffic(W.WORKLOADS["ctx_128k"])
+    assert t is None or abs(t - 136.3e6) < 1e5
