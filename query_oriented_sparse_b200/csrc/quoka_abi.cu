@@ -16,6 +16,7 @@
 #include "topk.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "attn_tc2.cuh"
 #include "compact.cuh"
 
 using namespace quoka;
@@ -320,6 +321,26 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
   CUtensorMap qmap, kmap, vmap;
   quoka_status s;
   if ((s = make_map_bf16(&qmap, q, (uint64_t)d.batch * d.h_q * d.C, D, 64, 1, "q_chunk")) != QUOKA_OK) return s;
+  if constexpr (D == 128) {
+    // SM pairs: each CTA loads 64-key halves of K tiles and 64-column halves of V tiles
+    if ((s = make_map_bf16(&kmap, kc, kc_rows, D, 64, 64, "compacted K")) != QUOKA_OK) return s;
+    if ((s = make_map_bf16(&vmap, vc, kc_rows, D, 64, 128, "compacted V")) != QUOKA_OK) return s;
+    Attn2Params p2;
+    p2.h_q = d.h_q;
+    p2.h_kv = d.h_kv;
+    p2.G = d.G;
+    p2.C = d.C;
+    p2.TP = p.TP;
+    p2.kc_stride = p.kc_stride;
+    p2.scale_log2 = p.scale_log2;
+    const int smem2 = At2Cfg::SMEM;
+    if ((e = ensure_smem(attn_tc2_kernel, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
+    dim3 grid2(2 * ((d.C + 2 * p.TP - 1) / (2 * p.TP)), d.h_kv, d.batch);
+    attn_tc2_kernel<<<grid2, AT2_THREADS, smem2, st>>>(qmap, kmap, vmap, tab, p2,
+                                                       reinterpret_cast<__nv_bfloat16*>(out));
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_tc2 launch");
+    return QUOKA_OK;
+  }
   if ((s = make_map_bf16(&kmap, kc, kc_rows, D, 64, 128, "compacted K")) != QUOKA_OK) return s;
   if ((s = make_map_bf16(&vmap, vc, kc_rows, D, 64, 128, "compacted V")) != QUOKA_OK) return s;
   const int smem = AtcCfg<D>::SMEM;
