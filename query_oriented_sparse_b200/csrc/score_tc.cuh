@@ -14,11 +14,10 @@
 // heads); its operand block stays resident in shared memory while key tiles stream
 // through a ring of 16 KB K-block stages loaded by TMA (128-byte swizzle).  Warp 0
 // issues TMA, one thread of warp 1 issues the MMAs of each tile as one or two column
-// slices (cut on head boundaries) into two 256-column TMEM accumulators, and two
-// epilogue warpgroups (warps 2-5 and 6-9) drain alternate accumulators, so every SM
-// sub-partition has two warps to interleave.  When a tile has two slices, the group
-// that drains the second one adds the other group's partial sum and |k|^2 share,
-// handed over through a shared-memory slot guarded by an mbarrier pair.
+// slices (cut on head boundaries) into two 256-column TMEM accumulators, and sixteen
+// epilogue warps in four groups drain them: group e takes the heads h with h % 4 == e
+// and a quarter of |k|^2, and groups 1-3 hand their partials to group 0 through a
+// shared-memory slot guarded by an mbarrier pair.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -28,7 +27,8 @@ constexpr int STC_BM = 128;        // keys per tile (TMEM lanes)
 constexpr int STC_MAXCOLS = 512;   // kept-query columns per column group
 constexpr int STC_SLICE = 256;     // max MMA N per accumulator slice
 constexpr int STC_NBUF = 2;        // accumulator slices held in TMEM
-constexpr int STC_THREADS = 320;   // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9 epilogue
+constexpr int STC_THREADS = 576;   // warp 0 TMA, warp 1 MMA, warps 2-17 epilogue (4 groups)
+constexpr int STC_EPI_WARPS = 16;
 constexpr int STC_QBOX = 16;       // rows per TMA box of the kept-query block
 
 struct ScoreTcParams {
@@ -54,7 +54,8 @@ struct StcCfg {
   // batch past a slice end still reads inside the arrays
   static constexpr int CP_BYTES = 2 * STC_MAXCOLS * 8;
   static constexpr int NBAR = 2 * NST + 2 + 2 * STC_NBUF + 4;
-  static constexpr int MERGE_BYTES = 2 * STC_BM * 8;   // two (partial sum, |k|^2 share) slots
+  // two slots of (partial sum, |k|^2 share) from epilogue groups 1-3
+  static constexpr int MERGE_BYTES = 2 * 3 * STC_BM * 8;
   static constexpr int SMEM = 1024 + Q_BYTES + K_BYTES + CP_BYTES + MERGE_BYTES + NBAR * 8 + 16;
 };
 
@@ -96,7 +97,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   uint64_t* qempty = qfull + 1;
   uint64_t* accfull = qfull + 2;
   uint64_t* accempty = accfull + STC_NBUF;
-  uint64_t* mfull = accempty + STC_NBUF;   // [2] partial sum of slice 0 written
+  uint64_t* mfull = accempty + STC_NBUF;   // [2] partials of groups 1-3 written
   uint64_t* mempty = mfull + 2;            // [2] slot consumed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
 
@@ -108,15 +109,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       ptx::mbar_init(&kfull[s], 1);
-      ptx::mbar_init(&kempty[s], 1 + 8);
+      ptx::mbar_init(&kempty[s], 1 + STC_EPI_WARPS);
     }
     ptx::mbar_init(qfull, 1);
     ptx::mbar_init(qempty, 1);
     for (int s = 0; s < STC_NBUF; ++s) {
       ptx::mbar_init(&accfull[s], 1);
-      ptx::mbar_init(&accempty[s], 4);
-      ptx::mbar_init(&mfull[s], 128);
-      ptx::mbar_init(&mempty[s], 128);
+      ptx::mbar_init(&accempty[s], STC_EPI_WARPS);
+      ptx::mbar_init(&mfull[s], 3 * STC_BM);
+      ptx::mbar_init(&mempty[s], STC_BM);
     }
     ptx::fence_mbar_init();
   }
@@ -223,11 +224,22 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       }
     }
   } else {
-    // ---------------- epilogue: two groups (warps 2-5, 6-9), one key per thread ----------
-    const int set = (warp - 2) >> 2;
+    // ---------------- epilogue: four groups of four warps, one key per thread ----------
+    // Group e (warps 2+4e .. 5+4e, one per TMEM lane quarter) takes the query heads h of
+    // the column group with h % 4 == e, so a head's columns never split across warps, and
+    // a quarter of the key's dimensions for |k|^2.  Groups 1-3 hand (sum of head maxima,
+    // |k|^2 share) to group 0 through a shared-memory slot, and group 0 adds them in group
+    // order and writes the pooled score.  Four warps per SM sub-partition interleave
+    // their TMEM loads, which a single warp cannot overlap with its own arithmetic.
+    const int e = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    constexpr int DQ = D / 4;                    // dimensions of |k|^2 per group
+    constexpr int CHUNKS = DQ / 8;               // 16-byte chunks (8 bf16) per group
+    const int kb_e = (e * DQ) / 64;              // K-block holding this group's dimensions
+    const int ch0 = ((e * DQ) % 64) / 8;         // first chunk of the 128-byte row
+    float2* mslot = reinterpret_cast<float2*>(merge);
     int stage = 0, cur = -1, nsl_done = 0, ncols = 0, nmerge = 0;
     uint32_t kph = 0;
     bool ok = true;
@@ -236,20 +248,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       stc_decode(p, tab, u, b, g, cg, tile);
       const int key3 = (b * p.h_kv + g) * p.ncg + cg;
       if (key3 != cur) {
-        ptx::named_bar(1, 256);
+        ptx::named_bar(1, 32 * STC_EPI_WARPS);
         const int h0 = cg * p.heads_per_cg;
         ncols = (min(p.G, h0 + p.heads_per_cg) - h0) * p.nkp;
         const size_t c0 = (size_t)(b * p.h_kv + g) * p.G * p.nkp + (size_t)h0 * p.nkp;
-        for (int c = threadIdx.x - 64; c < ncols; c += 256) {
+        for (int c = threadIdx.x - 64; c < ncols; c += 32 * STC_EPI_WARPS) {
           cpi[c] = qinv[c0 + c];
           cpb[c] = qbias[c0 + c];
         }
-        ptx::named_bar(1, 256);
+        ptx::named_bar(1, 32 * STC_EPI_WARPS);
         cur = key3;
       }
+      const int nh = ncols / p.nkp;                // query heads in this column group
       const int nsl = ncols > STC_SLICE ? 2 : 1;
-      const int cols0 = nsl == 2 ? ((ncols / p.nkp + 1) / 2) * p.nkp : ncols;
-      const int fin = (nsl_done + nsl - 1) & 1;   // group draining the tile's last slice
+      const int hs0 = nsl == 2 ? (nh + 1) / 2 : nh; // heads in slice 0 (head-aligned cut)
       int st[KB];
       uint32_t sph[KB];                            // ring slot and its phase per K-block
       for (int kb = 0; kb < KB; ++kb) {
@@ -257,30 +269,23 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         sph[kb] = kph;
         if (++stage == NST) { stage = 0; kph ^= 1u; }
       }
-      // |k|^2 of this thread's key from the swizzled tile in shared memory: the owner of
-      // a one-slice tile reads every K-block, a two-slice tile splits them
-      int kb_lo = 0, kb_hi = 0;
-      if (nsl == 1) {
-        if (set == fin) kb_hi = KB;
-      } else {
-        kb_lo = (set == fin) ? KB / 2 : 0;
-        kb_hi = (set == fin) ? KB : KB / 2;
-      }
-      float ss = 0.f;
-      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+      // Every K-block of the tile has landed before this warp releases it: a release of a
+      // slot this warp never waited for could otherwise count toward the slot's previous
+      // use.  Then |k|^2 over this group's dimensions from the swizzled tile.
+      for (int kb = 0; kb < KB; ++kb)
         if (ok) ok = ptx::mbar_wait(&kfull[st[kb]], sph[kb]);
-        if (ok) {
-          const uint8_t* rp = sK + st[kb] * Cfg::STAGE_BYTES + row * 128;
+      float ss = 0.f;
+      if (ok) {
+        const uint8_t* rp = sK + st[kb_e] * Cfg::STAGE_BYTES + row * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(rp + ((c ^ (row & 7)) << 4));
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        for (int c = 0; c < CHUNKS; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(rp + (((ch0 + c) ^ (row & 7)) << 4));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
-              ss = fmaf(lo, lo, ss);
-              ss = fmaf(hi, hi, ss);
-            }
+          for (int i = 0; i < 4; ++i) {
+            const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
+            ss = fmaf(lo, lo, ss);
+            ss = fmaf(hi, hi, ss);
           }
         }
       }
@@ -289,102 +294,88 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         for (int kb = 0; kb < KB; ++kb) ptx::mbar_arrive(&kempty[st[kb]]);
       if (!ok) break;
 
+      // sum over this group's heads of max over the head's kept queries of s / |q| (+ bias)
       float sum = 0.f;
       for (int sl = 0; sl < nsl && ok; ++sl, ++nsl_done) {
         const int buf = nsl_done & 1;
-        if (buf != set) continue;
         const uint32_t bph = (uint32_t)(nsl_done >> 1) & 1u;
+        // every group waits for every slice before releasing it, which keeps the
+        // accumulator's release barrier in step with its uses
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&accfull[buf], bph));
         if (!ok) break;
         ptx::tc_fence_after();
-        const int cbase = sl == 0 ? 0 : cols0;
-        const int nc = sl == 0 ? cols0 : ncols - cols0;
-        float run = -INFINITY;
-        int to_boundary = p.nkp;                 // columns left in the current head
-        for (int c0 = 0; c0 < nc; c0 += 64) {
-          // up to 64 columns of TMEM loads in flight per wait
-          uint32_t r[2][32];
+        const int h_lo = sl == 0 ? 0 : hs0, h_hi = sl == 0 ? hs0 : nh;
+        for (int h = h_lo + ((e - h_lo) & 3); h < h_hi; h += 4) {
+          const uint32_t tcol = (uint32_t)(buf * STC_SLICE + (h - h_lo) * p.nkp);
+          const float* ci = cpi + h * p.nkp;
+          const float* cb = cpb + h * p.nkp;
+          float run = -INFINITY;
+          for (int c = 0; c < p.nkp; c += 32) {
+            const int w = min(32, p.nkp - c);       // 32 or (odd tail) 16 columns
+            uint32_t r[32];
+            if (w == 32) ptx::tmem_ld32(lane_base + tcol + (uint32_t)c, r);
+            else ptx::tmem_ld16(lane_base + tcol + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(r));
+            ptx::tmem_ld_wait();
 #pragma unroll
-          for (int q4 = 0; q4 < 2; ++q4)
-            if (c0 + q4 * 32 < nc)
-              ptx::tmem_ld32(lane_base + (uint32_t)(buf * STC_SLICE + c0 + q4 * 32), r[q4]);
-          ptx::tmem_ld_wait();
-          // four independent 16-column maxima of (s * 1/|q| + bias); groups past the
-          // slice end are -inf.  Columns of a group always belong to one query head.
-          float gm[4];
-          const float4* ci4 = reinterpret_cast<const float4*>(cpi + cbase + c0);
-          const float4* cb4 = reinterpret_cast<const float4*>(cpb + cbase + c0);
+            for (int q = 0; q < 2; ++q) {
+              if (q * 16 < w) {
+                float v[16];
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            float v[16];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float4 sc = ci4[q8 * 4 + i];
-              const uint32_t* rr = &r[q8 >> 1][(q8 & 1) * 16 + 4 * i];
-              const float2 s01 = make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1]));
-              const float2 s23 = make_float2(__uint_as_float(rr[2]), __uint_as_float(rr[3]));
-              float2 v01, v23;
-              if (p.padded) {
-                const float4 bi = cb4[q8 * 4 + i];
-                v01 = ptx::fma2(s01, make_float2(sc.x, sc.y), make_float2(bi.x, bi.y));
-                v23 = ptx::fma2(s23, make_float2(sc.z, sc.w), make_float2(bi.z, bi.w));
-              } else {
-                v01 = ptx::mul2(s01, make_float2(sc.x, sc.y));
-                v23 = ptx::mul2(s23, make_float2(sc.z, sc.w));
+                for (int i = 0; i < 4; ++i) {
+                  const float4 sc = reinterpret_cast<const float4*>(ci + c + q * 16)[i];
+                  const uint32_t* rr = &r[q * 16 + 4 * i];
+                  const float2 s01 = make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1]));
+                  const float2 s23 = make_float2(__uint_as_float(rr[2]), __uint_as_float(rr[3]));
+                  float2 v01, v23;
+                  if (p.padded) {
+                    const float4 bi = reinterpret_cast<const float4*>(cb + c + q * 16)[i];
+                    v01 = ptx::fma2(s01, make_float2(sc.x, sc.y), make_float2(bi.x, bi.y));
+                    v23 = ptx::fma2(s23, make_float2(sc.z, sc.w), make_float2(bi.z, bi.w));
+                  } else {
+                    v01 = ptx::mul2(s01, make_float2(sc.x, sc.y));
+                    v23 = ptx::mul2(s23, make_float2(sc.z, sc.w));
+                  }
+                  v[4 * i] = v01.x; v[4 * i + 1] = v01.y; v[4 * i + 2] = v23.x; v[4 * i + 3] = v23.y;
+                }
+                const float a0 = ptx::max3(v[0], v[1], v[2]), a1 = ptx::max3(v[3], v[4], v[5]);
+                const float a2 = ptx::max3(v[6], v[7], v[8]), a3 = ptx::max3(v[9], v[10], v[11]);
+                const float a4 = ptx::max3(v[12], v[13], v[14]);
+                run = ptx::max3(run, ptx::max3(a0, a1, a2), ptx::max3(a3, a4, v[15]));
               }
-              v[4 * i] = v01.x; v[4 * i + 1] = v01.y; v[4 * i + 2] = v23.x; v[4 * i + 3] = v23.y;
-            }
-            const float a0 = ptx::max3(v[0], v[1], v[2]), a1 = ptx::max3(v[3], v[4], v[5]);
-            const float a2 = ptx::max3(v[6], v[7], v[8]), a3 = ptx::max3(v[9], v[10], v[11]);
-            const float a4 = ptx::max3(v[12], v[13], v[14]);
-            const float m = fmaxf(ptx::max3(a0, a1, a2), ptx::max3(a3, a4, v[15]));
-            gm[q8] = (c0 + q8 * 16 < nc) ? m : -INFINITY;
-          }
-          const int ng = min(4, (nc - c0) >> 4);
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            if (q8 < ng) {
-              if (to_boundary == 0) {              // a new query head starts here
-                sum += run;
-                run = -INFINITY;
-                to_boundary = p.nkp;
-              }
-              to_boundary -= 16;
-              run = fmaxf(run, gm[q8]);
             }
           }
+          sum += run;
         }
-        sum += run;
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&accempty[buf]);
       }
       if (!ok) break;
-      if (nsl == 2) {
-        const int slot = nmerge & 1;
-        const uint32_t mph = (uint32_t)(nmerge >> 1) & 1u;
-        ++nmerge;
-        if (set != fin) {                           // hand slice 0's partial sum over
-          ok = __all_sync(0xffffffffu, ptx::mbar_wait(&mempty[slot], mph ^ 1u));
-          if (!ok) break;
-          reinterpret_cast<float2*>(merge)[slot * STC_BM + row] = make_float2(sum, ss);
-          ptx::mbar_arrive(&mfull[slot]);
-          continue;
-        }
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&mfull[slot], mph));
+
+      const int slot = nmerge & 1;
+      const uint32_t mph = (uint32_t)(nmerge >> 1) & 1u;
+      ++nmerge;
+      if (e != 0) {                                // hand this group's partials to group 0
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&mempty[slot], mph ^ 1u));
         if (!ok) break;
-        const float2 other = reinterpret_cast<float2*>(merge)[slot * STC_BM + row];
-        sum = other.x + sum;
-        ss = other.y + ss;
-        ptx::mbar_arrive(&mempty[slot]);
-      } else if (set != fin) {
+        mslot[(slot * 3 + (e - 1)) * STC_BM + row] = make_float2(sum, ss);
+        ptx::mbar_arrive(&mfull[slot]);
         continue;
       }
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&mfull[slot], mph));
+      if (!ok) break;
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        const float2 o = mslot[(slot * 3 + q) * STC_BM + row];
+        sum += o.x;
+        ss += o.y;
+      }
+      ptx::mbar_arrive(&mempty[slot]);
       const float knorm = sqrtf(ss);
       const int j = tile * STC_BM + row;
       if (j < tab.prefix[b]) {
-        const float s = knorm > 0.f ? (p.ncg == 1 ? sum * p.inv_G : sum) / knorm : 0.f;
-        pooled[cg * p.cg_stride + (size_t)(b * p.h_kv + g) * p.pooled_stride + j] = s;
+        const float sc = knorm > 0.f ? (p.ncg == 1 ? sum * p.inv_G : sum) / knorm : 0.f;
+        pooled[cg * p.cg_stride + (size_t)(b * p.h_kv + g) * p.pooled_stride + j] = sc;
       }
     }
   }
