@@ -203,6 +203,21 @@ cudaError_t ensure_smem(K kernel, int bytes) {
   return e;
 }
 
+// Allows a kernel's clusters above the portable size of 8 CTAs (B200 schedules 16).
+template <typename K>
+cudaError_t ensure_cluster16(K kernel) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::map<std::pair<const void*, int>, bool> done;
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lock(g_smem_mu);
+  if (done.count(key)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) done[key] = true;
+  return e;
+}
+
 template <int D>
 quoka_status launch_score_tc(const Dims& d, const SeqTable& tab, long long rows, const void* k,
                              unsigned char* ws, const WsLayout& w, cudaStream_t st) {
@@ -275,6 +290,7 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
   const int tk_keys = std::min((tab.max_prefix + TOPK_CS - 1) / TOPK_CS, TOPK_STAGE_KEYS);
   const int tk_smem = tk_keys * 4;
   if ((e = ensure_smem(topk_kernel, tk_smem)) != cudaSuccess) return cuda_fail(e, "topk smem");
+  if ((e = ensure_cluster16(topk_kernel)) != cudaSuccess) return cuda_fail(e, "topk cluster size");
   topk_kernel<<<d.batch * d.h_kv * TOPK_CS, TOPK_THREADS, tk_smem, st>>>(
       pooled, w.pooled_stride, w.ncg, w.cg_stride, 1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");

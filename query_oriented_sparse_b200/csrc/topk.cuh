@@ -2,7 +2,7 @@
 // ascending index order (QUOKA page, Figure 1(a): the KV cache is sub-selected into a
 // compacted cache before dense attention).
 //
-// One thread-block cluster of TOPK_CS CTAs per (sequence, KV head); CTA r owns a
+// One thread-block cluster of TOPK_CS = 16 CTAs per (sequence, KV head); CTA r owns a
 // contiguous slice of the prefix.  The exact B-th largest score is found by a cluster
 // radix select over orderable score keys and the kept indices are emitted in index
 // order (cluster_select.cuh), so the result is deterministic and sorted without a sort.
@@ -16,7 +16,8 @@
 
 namespace quoka {
 
-constexpr int TOPK_CS = 8;
+constexpr int TOPK_CS = 16;                   // CTAs per (sequence, KV head); a non-portable
+                                              // cluster size, opted into at launch
 constexpr int TOPK_THREADS = 512;
 constexpr int TOPK_STAGE_KEYS = 49152;         // keys staged per CTA (192 KB)
 
