@@ -177,12 +177,10 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       const uint32_t q_lo = (uint32_t)q_d, q_hi = (uint32_t)(q_d >> 32);
       const uint32_t k_lo = (uint32_t)k_d, k_hi = (uint32_t)(k_d >> 32);
       const uint32_t v_lo = (uint32_t)v_d, v_hi = (uint32_t)(v_d >> 32);
-      // S(j) into buffer j % 2 (columns 128 * (j % 2)), once block j's K and V have landed
-      // in both CTAs (P.V(j) later reads V(j) from the same stage without another wait)
-      auto issue_s = [&](int j) -> bool {
+      // S(j) into buffer j % 2 (columns 128 * (j % 2)); block j's K and V have landed in
+      // both CTAs (P.V(j) later reads V(j) from the same stage without another wait)
+      auto s_mmas = [&](int j) {
         const int st = j % AT2_ST;
-        if (!ptx::mbar_wait_cluster(&kvfull[st], (uint32_t)(j / AT2_ST) & 1u)) return false;
-        ptx::tc_fence_after();
         const uint32_t b0 = k_lo + (uint32_t)(st * (Cfg::KH_BYTES >> 4));
         const uint32_t d = tmem + (uint32_t)((j & 1) * 128);
 #pragma unroll
@@ -191,15 +189,27 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
           for (int k = 0; k < 4; ++k)
             ptx::mma_bf16_ss_pair(d, q_lo + (uint32_t)(kb * 1024 + k * 2), q_hi,
                                   b0 + (uint32_t)(kb * 512 + k * 2), k_hi, idesc_s, (kb | k) ? 1u : 0u);
-        ptx::tc_commit_pair(&sfull[j & 1], kBoth);
-        return true;
+      };
+      auto kv_landed = [&](int j) -> bool {
+        return ptx::mbar_wait_cluster(&kvfull[j % AT2_ST], (uint32_t)(j / AT2_ST) & 1u);
       };
       bool ok = ptx::mbar_wait(qfull, 0) && ptx::mbar_wait_cluster(qpeer, 0);
-      if (ok) ok = issue_s(0);
-      if (ok && nblk > 1) ok = issue_s(1);
+      for (int j = 0; j < 2 && j < nblk && ok; ++j) {
+        ok = kv_landed(j);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        s_mmas(j);
+        ptx::tc_commit_pair(&sfull[j & 1], kBoth);
+      }
+      // Per block: every wait comes before the block's 16 MMAs, which are issued back to
+      // back (a wait or commit between them lets the tensor pipe's short queue drain), and
+      // both commits come after them.  The stage of block j is released once S(j+2) is
+      // done, which also implies P.V(j) is.
       for (int j = 0; j < nblk && ok; ++j) {
         const int st = j % AT2_ST;
-        ok = ptx::mbar_wait_cluster(&pready[j & 1], (uint32_t)(j >> 1) & 1u);
+        const bool more = j + 2 < nblk;
+        if (more) ok = kv_landed(j + 2);
+        if (ok) ok = ptx::mbar_wait_cluster(&pready[j & 1], (uint32_t)(j >> 1) & 1u);
         if (!ok) break;
         ptx::tc_fence_after();
         // O += P(j) V(j); P(j) lies in buffer j % 2: keys 0-63 in columns 0-31, keys
@@ -210,8 +220,11 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         for (int k = 0; k < 8; ++k)
           ptx::mma_bf16_ts_pair(tmem + 256u, pa + (uint32_t)(k < 4 ? k * 8 : 96 + (k - 4) * 8),
                                 b0 + (uint32_t)(k * 128), v_hi, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+        if (more) {
+          s_mmas(j + 2);
+          ptx::tc_commit_pair(&sfull[j & 1], kBoth);
+        }
         ptx::tc_commit_pair(&kvempty[st], kBoth);
-        if (j + 2 < nblk) ok = issue_s(j + 2);
       }
     }
   } else {
