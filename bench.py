@@ -38,10 +38,10 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 LAUNCHES_PER_STEP = 5  # qsub, score, top-k, compaction, attention
 # DRAM traffic of one attention-kernel launch on the 128K-context workload
 # (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture, summarised in
-# profiles/attn_tc_kernel_ctx_128k.md), valid only for the kernel sources it was taken
+# profiles/attn_tc2_kernel_ctx_128k.md), valid only for the kernel sources it was taken
 # on: the digest below covers them, and a changed kernel reports null.
-ATTN_TRAFFIC = {"workload": "ctx_128k", "bytes": 117.492992e6 + 18.832384e6,
-                "sources": ['query_oriented_sparse_b200/csrc/attn_tc.cuh', 'query_oriented_sparse_b200/csrc/tc_ptx.cuh'], "sha256_16": "74f457a2a89ca874"}
+ATTN_TRAFFIC = {"workload": "ctx_128k", "bytes": 117.495040e6 + 19.681024e6,
+                "sources": ['query_oriented_sparse_b200/csrc/attn_tc2.cuh', 'query_oriented_sparse_b200/csrc/tc_ptx.cuh'], "sha256_16": "b59e03c2044e38e6"}
 
 
 def attn_traffic(w):
@@ -397,7 +397,7 @@ def run_ours(args, w):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                      "traffic": attn_traffic(w),
-                     "kernel": "attn_tc_kernel, timed as the sparse_chunk_attn call (compaction + attention)",
+                     "kernel": "attn_tc2_kernel (SM pairs), timed as the sparse_chunk_attn call (compaction + attention)",
                      "peak_source": f"{peak_src} bf16 dense (burst)"},
         "path_roofline": {"roofline_us": path_roof_us, "stage_roofline_us": rl,
                           "measured_us": total_s * 1e6 / args.steps,
