@@ -73,32 +73,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
   }
 }
-// Non-suspending probe of a phase, cluster-scope acquire.
-__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded polling wait for barriers that other SMs complete (remote arrivals, multicast
-// commits, another CTA's TMA bytes): test_wait never suspends the thread, so the phase
-// is seen as soon as it completes.
-__device__ __forceinline__ bool mbar_poll_cluster(uint64_t* bar, uint32_t parity) {
-  if (mbar_test_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_test_wait_cluster(bar, parity)) return true;
-    if ((i & 1023u) == 0 && globaltimer() - t0 > kWaitLimitNs) {
-      flag_error(ERR_WAIT_TIMEOUT);
-      return false;
-    }
-  }
-}
 // As mbar_wait, with cluster-scope acquire.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
