@@ -1,5 +1,5 @@
 // Shared device-side helpers of libquoka: element types, the per-call sequence table,
-// orderable float keys, block-wide scans and the device error word.
+// orderable float keys, warp reductions and the device error word.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -86,43 +86,12 @@ __device__ __forceinline__ uint32_t float_to_ordered(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// ---- warp / block helpers --------------------------------------------------------
+// ---- warp helpers --------------------------------------------------------
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
-}
-
-// Exclusive block scan of one int flag/count per thread; returns the thread's
-// exclusive prefix and writes the block total to *total.  `scratch` holds at least
-// (blockDim.x / 32 + 1) ints.  Must be called by every thread of the block.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) scratch[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = (lane < nwarps) ? scratch[lane] : 0;
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += y;
-    }
-    if (lane < nwarps) scratch[lane] = wi - w;  // exclusive warp offsets
-    if (lane == nwarps - 1) scratch[32] = wi;
-  }
-  __syncthreads();
-  int res = scratch[warp] + incl - v;
-  *total = scratch[32];
-  __syncthreads();
-  return res;
 }
 
 }  // namespace quoka

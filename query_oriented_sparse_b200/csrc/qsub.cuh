@@ -3,16 +3,23 @@
 // from the mean interact with more keys).
 //
 // One thread-block cluster of QSUB_CS CTAs per (sequence, query head); CTA r owns a
-// contiguous slice of the chunk positions.  Pass 1 streams the slice once with vector
-// loads (eight rows in flight per warp), takes |q_t| with a warp reduction and sums the
-// unit queries; the CTAs' partial sums meet through distributed shared memory (in rank
-// order, so the mean direction is the same on every CTA).  Pass 2 re-reads the slice
-// (L2-resident) for c_t = cos(q_t, mean) as orderable keys in shared memory.  A cluster
-// radix select keeps the Nk smallest, ties to the lower t, in ascending t
-// (cluster_select.cuh).  The kept rows are copied (raw values) into the per-KV-head
-// operand block of the scoring GEMM with their fp32 1/|q| and a column bias; each
-// head's block is padded to nkp rows (a multiple of 16) with zero rows whose bias is
-// -inf, so a padded column can never win the max pooling.
+// contiguous slice of the chunk positions.  Rows are read eight lanes to a row (a warp
+// takes four rows per step, each lane one or more 16-byte vectors), several steps in
+// flight per warp, so a row's reductions are three shuffles wide instead of a serial
+// five-shuffle chain per row.
+//   pass 1  |q_t| and the sum of unit queries over this CTA's slice; the CTAs' partial
+//           sums meet through distributed shared memory (in rank order, so the mean
+//           direction is the same on every CTA);
+//   pass 2  re-reads the slice (L2-resident) for c_t = cos(q_t, mean) as orderable keys,
+//           stored at their chunk position in a chunk-wide key array;
+//   select  after one cluster barrier every CTA copies the other CTAs' keys into its own
+//           array (the whole chunk is at most 32 KB of keys) and runs the radix select of
+//           the Nk smallest (ties to the lower t) locally, with block barriers only
+//           (cluster_select.cuh); each CTA emits the kept positions of its own slice.
+// The kept rows are copied (raw values) into the per-KV-head operand block of the scoring
+// GEMM with their fp32 1/|q| and a column bias; each head's block is padded to nkp rows
+// (a multiple of 16) with zero rows whose bias is -inf, so a padded column can never win
+// the max pooling.
 #pragma once
 #include "cluster_select.cuh"
 
@@ -22,60 +29,132 @@ constexpr int QSUB_CS = 8;                    // CTAs per query head
 constexpr int QSUB_THREADS = 512;
 constexpr int QSUB_WARPS = QSUB_THREADS / 32;
 constexpr int QSUB_MAX_ROWS = (QUOKA_MAX_CHUNK + QSUB_CS - 1) / QSUB_CS;
-constexpr int QSUB_UNROLL = 8;
+constexpr int QSUB_LPR = 8;                   // lanes per query row
+constexpr int QSUB_RPS = 32 / QSUB_LPR;       // rows per warp step
+
+// Per-lane view of a row: NV 16-byte vectors, vector v of lane l8 holding elements
+// [(8 v + l8) VE, (8 v + l8 + 1) VE).  U steps are in flight per warp (16 registers of
+// raw row data per lane, which keeps two 512-thread CTAs per SM without spills).
+template <typename T, int D>
+struct QsubShape {
+  static constexpr int VE = 16 / (int)sizeof(T);
+  static constexpr int NV = D / (QSUB_LPR * VE);
+  static constexpr int EPL = NV * VE;
+  static constexpr int U = NV >= 4 ? 1 : 4 / NV;
+  static_assert(NV * QSUB_LPR * VE == D, "row width must be a multiple of 8 vectors");
+};
+
+template <typename T> struct Unpack;
+template <> struct Unpack<__nv_bfloat16> {
+  __device__ static __forceinline__ void run(const uint4& r, float* x) {
+    const unsigned int w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      unsigned int wi = w[i];
+      const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wi));
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+};
+template <> struct Unpack<float> {
+  __device__ static __forceinline__ void run(const uint4& r, float* x) {
+    x[0] = __uint_as_float(r.x); x[1] = __uint_as_float(r.y);
+    x[2] = __uint_as_float(r.z); x[3] = __uint_as_float(r.w);
+  }
+};
+
+__device__ __forceinline__ float group8_sum(float v) {   // sum over the 8 lanes of a row
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
+  return v;
+}
 
 template <typename T, int D>
-__global__ void __cluster_dims__(QSUB_CS, 1, 1) __launch_bounds__(QSUB_THREADS)
+__global__ void __cluster_dims__(QSUB_CS, 1, 1) __launch_bounds__(QSUB_THREADS, 2)
 qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
             int32_t* __restrict__ kept_out, T* __restrict__ qsel, float* __restrict__ qinv,
             float* __restrict__ qbias) {
-  constexpr int PER = D / 32;                 // elements per lane per row
+  using Sh = QsubShape<T, D>;
+  constexpr int VE = Sh::VE, NV = Sh::NV, EPL = Sh::EPL, U = Sh::U;
   cg::cluster_group cluster = cg::this_cluster();
   __shared__ float inv[QSUB_MAX_ROWS];
-  __shared__ uint32_t keys[QSUB_MAX_ROWS];
   __shared__ float part[QSUB_WARPS][D];
   __shared__ float cta_sum[D];
   __shared__ float mdir[D];
   __shared__ float mscale_s;
-  __shared__ ClusterSelectSmem sm;
+  __shared__ SelectSmem sm;
   __shared__ int kept_pos[QSUB_MAX_ROWS], kept_t[QSUB_MAX_ROWS];
   __shared__ int n_kept;
+  extern __shared__ uint32_t keys[];          // C entries: c_t keys at chunk position t
 
   const int rank = (int)cluster.block_rank();
   const int bh = blockIdx.x / QSUB_CS;        // b * h_q + h
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 3, l8 = lane & 7;
   const int S = (C + QSUB_CS - 1) / QSUB_CS;
   const int lo = min(C, rank * S), hi = min(C, lo + S);
+  const int n = hi - lo;
   const T* qh = q + (size_t)bh * C * D;
 
-  // pass 1: norms and the sum of unit queries over this CTA's slice
-  float acc[PER];
+  // Row step u of this CTA covers rows lo + 4u .. lo + 4u + 3; warp w takes steps
+  // w, w + 16, ...; lanes beyond the slice load zeros and take part in the shuffles.
+  auto load_steps = [&](int u0, uint4 (&raw)[U][NV]) {
 #pragma unroll
-  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  for (int t0 = lo + warp; t0 < hi; t0 += QSUB_WARPS * QSUB_UNROLL) {
-    float x[QSUB_UNROLL][PER];
+    for (int i = 0; i < U; ++i) {
+      const int r = (u0 + i * QSUB_WARPS) * QSUB_RPS + g;
+      const uint4* src = reinterpret_cast<const uint4*>(qh + (size_t)(lo + r) * D);
 #pragma unroll
-    for (int u = 0; u < QSUB_UNROLL; ++u) {
-      const int t = t0 + u * QSUB_WARPS;
-      if (t < hi) load_vec<T, PER>(qh + (size_t)t * D + lane * PER, x[u]);
+      for (int v = 0; v < NV; ++v)
+        raw[i][v] = r < n ? __ldg(src + v * QSUB_LPR + l8) : make_uint4(0u, 0u, 0u, 0u);
     }
+  };
+
+  // pass 1: norms and the sum of unit queries over this CTA's slice
+  float acc[EPL];
 #pragma unroll
-    for (int u = 0; u < QSUB_UNROLL; ++u) {
-      const int t = t0 + u * QSUB_WARPS;
-      if (t >= hi) break;
+  for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+  for (int u0 = warp; u0 * QSUB_RPS < n; u0 += QSUB_WARPS * U) {
+    uint4 raw[U][NV];
+    load_steps(u0, raw);
+#pragma unroll
+    for (int i = 0; i < U; ++i) {
+      const int r = (u0 + i * QSUB_WARPS) * QSUB_RPS + g;
       float ss = 0.f;
 #pragma unroll
-      for (int i = 0; i < PER; ++i) ss = fmaf(x[u][i], x[u][i], ss);
-      ss = warp_sum(ss);
-      const float n = sqrtf(ss);
-      const float iv = n > 0.f ? 1.0f / n : 0.f;
+      for (int v = 0; v < NV; ++v) {
+        float x[VE];
+        Unpack<T>::run(raw[i][v], x);
 #pragma unroll
-      for (int i = 0; i < PER; ++i) acc[i] = fmaf(x[u][i], iv, acc[i]);
-      if (lane == 0) inv[t - lo] = iv;
+        for (int e = 0; e < VE; ++e) ss = fmaf(x[e], x[e], ss);
+      }
+      ss = group8_sum(ss);
+      const float nrm = sqrtf(ss);
+      const float iv = nrm > 0.f ? 1.0f / nrm : 0.f;
+      if (r < n) {
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          float x[VE];
+          Unpack<T>::run(raw[i][v], x);
+#pragma unroll
+          for (int e = 0; e < VE; ++e) acc[v * VE + e] = fmaf(x[e], iv, acc[v * VE + e]);
+        }
+        if (l8 == 0) inv[r] = iv;
+      }
     }
   }
 #pragma unroll
-  for (int i = 0; i < PER; ++i) part[warp][lane * PER + i] = acc[i];
+  for (int e = 0; e < EPL; ++e) {             // the warp's four row groups, fixed order
+    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+  }
+  if (g == 0) {
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+#pragma unroll
+      for (int e = 0; e < VE; ++e) part[warp][(v * QSUB_LPR + l8) * VE + e] = acc[v * VE + e];
+  }
   __syncthreads();
   if (tid < D) {
     float s = 0.f;
@@ -90,7 +169,8 @@ qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
     for (int r = 0; r < QSUB_CS; ++r) s += cluster.map_shared_rank(cta_sum, r)[tid];
     mdir[tid] = s;
   }
-  cluster.sync();                              // remote reads done before anyone moves on
+  cluster_arrive();                            // remote reads of cta_sum done; waited below
+  __syncthreads();
   if (warp == 0) {
     float s = 0.f;
     for (int d = lane; d < D; d += 32) s = fmaf(mdir[d], mdir[d], s);
@@ -101,34 +181,37 @@ qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
   const float mscale = mscale_s;
 
   // pass 2: c_t = (q_t . m) / (|q_t| |m|) as ascending-orderable keys
-  float mv[PER];
+  float mv[EPL];
 #pragma unroll
-  for (int i = 0; i < PER; ++i) mv[i] = mdir[lane * PER + i];
-  for (int t0 = lo + warp; t0 < hi; t0 += QSUB_WARPS * QSUB_UNROLL) {
-    float x[QSUB_UNROLL][PER];
+  for (int v = 0; v < NV; ++v)
 #pragma unroll
-    for (int u = 0; u < QSUB_UNROLL; ++u) {
-      const int t = t0 + u * QSUB_WARPS;
-      if (t < hi) load_vec<T, PER>(qh + (size_t)t * D + lane * PER, x[u]);
-    }
+    for (int e = 0; e < VE; ++e) mv[v * VE + e] = mdir[(v * QSUB_LPR + l8) * VE + e];
+  for (int u0 = warp; u0 * QSUB_RPS < n; u0 += QSUB_WARPS * U) {
+    uint4 raw[U][NV];
+    load_steps(u0, raw);
 #pragma unroll
-    for (int u = 0; u < QSUB_UNROLL; ++u) {
-      const int t = t0 + u * QSUB_WARPS;
-      if (t >= hi) break;
+    for (int i = 0; i < U; ++i) {
+      const int r = (u0 + i * QSUB_WARPS) * QSUB_RPS + g;
       float dot = 0.f;
 #pragma unroll
-      for (int i = 0; i < PER; ++i) dot = fmaf(x[u][i], mv[i], dot);
-      dot = warp_sum(dot);
-      if (lane == 0) keys[t - lo] = float_to_ordered(dot * inv[t - lo] * mscale);
+      for (int v = 0; v < NV; ++v) {
+        float x[VE];
+        Unpack<T>::run(raw[i][v], x);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) dot = fmaf(x[e], mv[v * VE + e], dot);
+      }
+      dot = group8_sum(dot);
+      if (r < n && l8 == 0) keys[lo + r] = float_to_ordered(dot * inv[r] * mscale);
     }
   }
-  __syncthreads();
+  cluster_wait();
 
   // keep the nk smallest (all of them when nk >= C), emitted in ascending t
   const size_t row0 = (size_t)bh * nkp;       // == ((b*h_kv + g)*G + h%G) * nkp
   if (tid == 0) n_kept = 0;
   __syncthreads();
   auto emit = [&](int pos, int t) {
+    if (t < lo || t >= hi) return;            // another CTA's position
     if (pos >= nk) { flag_error(ERR_BAD_INDEX); return; }   // unreachable when counts agree
     qinv[row0 + pos] = inv[t - lo];
     qbias[row0 + pos] = 0.f;
@@ -137,20 +220,26 @@ qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
     kept_pos[slot] = pos;
     kept_t[slot] = t;
   };
-  if (nk >= C) {
+  const bool select = nk < C;
+  if (!select) {
     for (int t = lo + tid; t < hi; t += blockDim.x) emit(t, t);
   } else {
-    auto key_at = [&](int j) { return keys[j - lo]; };
-    uint32_t thr;
-    int need_eq;
-    cluster_threshold<QSUB_CS, false>(cluster, sm, key_at, lo, hi, nk, &thr, &need_eq);
-    cluster_emit<QSUB_CS, false>(cluster, sm, key_at, lo, hi, thr, need_eq, emit);
+    cluster.sync();                            // every CTA's keys are final
+    for (int t = tid; t < C; t += blockDim.x) {
+      const int owner = t / S;
+      if (owner != rank) keys[t] = cluster.map_shared_rank(keys, owner)[t];
+    }
+    cluster_arrive();                          // remote reads of keys done; waited at the end
+    __syncthreads();
+    auto key_at = [&](int j) { return keys[j]; };
+    const SelectThreshold th = block_threshold<false>(sm, key_at, C, nk);
+    ordered_emit<false>(sm, key_at, 0, C, th, emit);
   }
   __syncthreads();
   {
     constexpr int VPR = D * (int)sizeof(T) / 16;   // 16-byte vectors per row
-    const int n = n_kept;
-    for (int e = tid; e < n * VPR; e += blockDim.x) {
+    const int nr = n_kept;
+    for (int e = tid; e < nr * VPR; e += blockDim.x) {
       const int i = e / VPR, v = e - i * VPR;
       const uint4* src = reinterpret_cast<const uint4*>(qh + (size_t)kept_t[i] * D);
       reinterpret_cast<uint4*>(qsel + (row0 + kept_pos[i]) * D)[v] = __ldg(src + v);
@@ -168,6 +257,7 @@ qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
     if (kept_out)
       for (int i = nk + tid; i < nq; i += blockDim.x) kept_out[(size_t)bh * nq + i] = -1;
   }
+  if (select) cluster_wait();                  // peers' last reads of this CTA's keys
 }
 
 }  // namespace quoka

@@ -268,7 +268,9 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
   float* pooled = reinterpret_cast<float*>(ws + w.pooled);
   cudaError_t e;
 
-  qsub_kernel<T, D><<<d.batch * d.h_q * QSUB_CS, QSUB_THREADS, 0, st>>>(
+  const int qs_smem = d.C * 4;                 // the chunk-wide key array
+  if ((e = ensure_smem(qsub_kernel<T, D>, qs_smem)) != cudaSuccess) return cuda_fail(e, "qsub smem");
+  qsub_kernel<T, D><<<d.batch * d.h_q * QSUB_CS, QSUB_THREADS, qs_smem, st>>>(
       reinterpret_cast<const T*>(q), d.C, w.nk, w.nkp, nq, kept_out, qsel, qinv, qbias);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "qsub launch");
 

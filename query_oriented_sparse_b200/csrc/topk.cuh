@@ -6,9 +6,9 @@
 // contiguous slice of the prefix.  The exact B-th largest score is found by a cluster
 // radix select over orderable score keys and the kept indices are emitted in index
 // order (cluster_select.cuh), so the result is deterministic and sorted without a sort.
-// Each CTA first stages its slice's keys in shared memory (coalesced, many loads in
-// flight), so the radix passes never wait on L2; slices longer than the staging area
-// read their keys from global memory instead.
+// Each CTA first stages its slice's keys in shared memory (coalesced, sixteen loads in
+// flight per thread), so the radix passes never wait on L2; slices longer than the
+// staging area read their keys from global memory instead.
 // When the scoring kernel split a KV head's kept queries into several column groups, a
 // first pass adds the groups' partial sums (in group order) and applies 1/G.
 #pragma once
@@ -20,13 +20,14 @@ constexpr int TOPK_CS = 16;                   // CTAs per (sequence, KV head); a
                                               // cluster size, opted into at launch
 constexpr int TOPK_THREADS = 512;
 constexpr int TOPK_STAGE_KEYS = 49152;         // keys staged per CTA (192 KB)
+constexpr int TOPK_STAGE_UNROLL = 16;          // staging loads in flight per thread
 
 __global__ void __cluster_dims__(TOPK_CS, 1, 1) __launch_bounds__(TOPK_THREADS)
 topk_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, long long cg_stride,
             float inv_G, const __grid_constant__ SeqTable tab, int h_kv, int b_max,
             int32_t* __restrict__ idx_out) {
   cg::cluster_group cluster = cg::this_cluster();
-  __shared__ ClusterSelectSmem sm;
+  __shared__ SelectSmem sm;
   extern __shared__ uint32_t staged[];         // TOPK_STAGE_KEYS entries when used
 
   const int rank = (int)cluster.block_rank();
@@ -60,31 +61,30 @@ topk_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, long l
     if (pos < B) out[pos] = j;
     else flag_error(ERR_BAD_INDEX);            // unreachable when the counts are consistent
   };
-  uint32_t thr;
-  int need_eq;
   if (hi - lo <= TOPK_STAGE_KEYS) {
-    for (int j0 = lo + threadIdx.x; j0 < hi; j0 += 4 * blockDim.x) {
-      float v[4];
+    for (int j0 = lo + threadIdx.x; j0 < hi; j0 += TOPK_STAGE_UNROLL * blockDim.x) {
+      float v[TOPK_STAGE_UNROLL];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < TOPK_STAGE_UNROLL; ++u) {
         const int j = j0 + u * blockDim.x;
         v[u] = j < hi ? sc[j] : 0.f;
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < TOPK_STAGE_UNROLL; ++u) {
         const int j = j0 + u * blockDim.x;
         if (j < hi) staged[j - lo] = float_to_ordered(v[u]);
       }
     }
     __syncthreads();
     auto key_at = [&](int j) { return staged[j - lo]; };
-    cluster_threshold<TOPK_CS, true>(cluster, sm, key_at, lo, hi, B, &thr, &need_eq);
-    cluster_emit<TOPK_CS, true>(cluster, sm, key_at, lo, hi, thr, need_eq, emit);
+    const SelectThreshold th = cluster_threshold<TOPK_CS, true>(cluster, sm, key_at, lo, hi, B);
+    ordered_emit<true>(sm, key_at, lo, hi, th, emit);
   } else {
     auto key_at = [sc](int j) { return float_to_ordered(sc[j]); };
-    cluster_threshold<TOPK_CS, true>(cluster, sm, key_at, lo, hi, B, &thr, &need_eq);
-    cluster_emit<TOPK_CS, true>(cluster, sm, key_at, lo, hi, thr, need_eq, emit);
+    const SelectThreshold th = cluster_threshold<TOPK_CS, true>(cluster, sm, key_at, lo, hi, B);
+    ordered_emit<true>(sm, key_at, lo, hi, th, emit);
   }
+  cluster_wait();                              // peers' last reads of this CTA's histograms
 }
 
 }  // namespace quoka
