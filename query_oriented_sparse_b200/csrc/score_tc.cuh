@@ -16,8 +16,10 @@
 // issues TMA, one thread of warp 1 issues the MMAs of each tile as one or two column
 // slices (cut on head boundaries) into two 256-column TMEM accumulators, and sixteen
 // epilogue warps in four groups drain them: group e takes the heads h with h % 4 == e
-// and a quarter of |k|^2, and groups 1-3 hand their partials to group 0 through a
-// shared-memory slot guarded by an mbarrier pair.
+// and a quarter of |k|^2.  After a tile every group hands (sum of its head maxima, |k|^2
+// share) to the tile's merging group (rotating over the tiles) through a shared-memory
+// slot guarded by an mbarrier pair; the merge runs one tile late, so no group waits for
+// the slowest one.  Waiting threads sleep on their mbarrier instead of spinning.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -54,8 +56,8 @@ struct StcCfg {
   // batch past a slice end still reads inside the arrays
   static constexpr int CP_BYTES = 2 * STC_MAXCOLS * 8;
   static constexpr int NBAR = 2 * NST + 2 + 2 * STC_NBUF + 4;
-  // two slots of (partial sum, |k|^2 share) from epilogue groups 1-3
-  static constexpr int MERGE_BYTES = 2 * 3 * STC_BM * 8;
+  // two slots of (partial sum, |k|^2 share) per epilogue group
+  static constexpr int MERGE_BYTES = 2 * 4 * STC_BM * 8;
   static constexpr int SMEM = 1024 + Q_BYTES + K_BYTES + CP_BYTES + MERGE_BYTES + NBAR * 8 + 16;
 };
 
@@ -69,6 +71,22 @@ __device__ __forceinline__ void stc_decode(const ScoreTcParams& p, const SeqTabl
   tile = rem - gc * tiles;
   g = gc / p.ncg;
   cg = gc - g * p.ncg;
+}
+
+// The unit after (b, g, cg, tile): a CTA walks a contiguous run of units, so after one
+// stc_decode it steps without divisions or indexed reads of the sequence table.
+__device__ __forceinline__ void stc_next(const ScoreTcParams& p, const SeqTable& tab, int& b,
+                                         int& g, int& cg, int& tile, int& tiles) {
+  if (++tile < tiles) return;
+  tile = 0;
+  if (++cg < p.ncg) return;
+  cg = 0;
+  if (++g < p.h_kv) return;
+  g = 0;
+  do {                                         // sequences without prefix keys own no units
+    ++b;
+    tiles = b < tab.batch ? (tab.prefix[b] + STC_BM - 1) / STC_BM : 1;
+  } while (tiles == 0);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -97,7 +115,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   uint64_t* qempty = qfull + 1;
   uint64_t* accfull = qfull + 2;
   uint64_t* accempty = accfull + STC_NBUF;
-  uint64_t* mfull = accempty + STC_NBUF;   // [2] partials of groups 1-3 written
+  uint64_t* mfull = accempty + STC_NBUF;   // [2] partials of all four groups written
   uint64_t* mempty = mfull + 2;            // [2] slot consumed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
 
@@ -116,7 +134,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     for (int s = 0; s < STC_NBUF; ++s) {
       ptx::mbar_init(&accfull[s], 1);
       ptx::mbar_init(&accempty[s], STC_EPI_WARPS);
-      ptx::mbar_init(&mfull[s], 3 * STC_BM);
+      ptx::mbar_init(&mfull[s], 4 * STC_BM);
       ptx::mbar_init(&mempty[s], STC_BM);
     }
     ptx::fence_mbar_init();
@@ -138,13 +156,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       int stage = 0, cur = -1;
       uint32_t kph = 0, qeph = 0;
       bool ok = true;
+      int b, g, cg, tile, tiles;
+      stc_decode(p, tab, u_lo, b, g, cg, tile);
+      tiles = (tab.prefix[b] + STC_BM - 1) / STC_BM;
       for (int u = u_lo; u < u_hi && ok; ++u) {
-        int b, g, cg, tile;
-        stc_decode(p, tab, u, b, g, cg, tile);
+        if (u != u_lo) stc_next(p, tab, b, g, cg, tile, tiles);
         const int key3 = (b * p.h_kv + g) * p.ncg + cg;
         if (key3 != cur) {
           if (cur >= 0) {
-            ok = ptx::mbar_wait(qempty, qeph);
+            ok = ptx::mbar_wait_sleep(qempty, qeph);
             qeph ^= 1u;
             if (!ok) break;
           }
@@ -160,7 +180,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         }
         const int krow = (int)(g * p.rows_per_head + tab.kv_off[b]) + tile * STC_BM;
         for (int kb = 0; kb < KB && ok; ++kb) {
-          ok = ptx::mbar_wait(&kempty[stage], kph ^ 1u);
+          ok = ptx::mbar_wait_sleep(&kempty[stage], kph ^ 1u);
           if (!ok) break;
           ptx::mbar_expect_tx(&kfull[stage], Cfg::STAGE_BYTES);
           ptx::tma_load_2d(sK + stage * Cfg::STAGE_BYTES, &kmap, &kfull[stage], kb * 64, krow);
@@ -174,13 +194,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       int stage = 0, cur = -1, nsl_done = 0, ncols = 0;
       uint32_t kph = 0, qph = 0;
       bool ok = true;
+      int b, g, cg, tile, tiles;
+      stc_decode(p, tab, u_lo, b, g, cg, tile);
+      tiles = (tab.prefix[b] + STC_BM - 1) / STC_BM;
       for (int u = u_lo; u < u_hi && ok; ++u) {
-        int b, g, cg, tile;
-        stc_decode(p, tab, u, b, g, cg, tile);
+        if (u != u_lo) stc_next(p, tab, b, g, cg, tile, tiles);
         const int key3 = (b * p.h_kv + g) * p.ncg + cg;
         if (key3 != cur) {
           if (cur >= 0) ptx::tc_commit(qempty);
-          ok = ptx::mbar_wait(qfull, qph);
+          ok = ptx::mbar_wait_sleep(qfull, qph);
           qph ^= 1u;
           if (!ok) break;
           const int h0 = cg * p.heads_per_cg;
@@ -190,7 +212,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         int st[KB];
         for (int kb = 0; kb < KB; ++kb) {
           st[kb] = stage;
-          if (ok) ok = ptx::mbar_wait(&kfull[stage], kph);
+          if (ok) ok = ptx::mbar_wait_sleep(&kfull[stage], kph);
           if (++stage == NST) { stage = 0; kph ^= 1u; }
         }
         if (!ok) break;
@@ -200,7 +222,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         for (int sl = 0; sl < nsl && ok; ++sl, ++nsl_done) {
           const int buf = nsl_done & 1;
           const uint32_t bph = (uint32_t)(nsl_done >> 1) & 1u;
-          ok = ptx::mbar_wait(&accempty[buf], bph ^ 1u);
+          ok = ptx::mbar_wait_sleep(&accempty[buf], bph ^ 1u);
           if (!ok) break;
           ptx::tc_fence_after();
           const int c0 = sl == 0 ? 0 : cols0;
@@ -226,11 +248,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   } else {
     // ---------------- epilogue: four groups of four warps, one key per thread ----------
     // Group e (warps 2+4e .. 5+4e, one per TMEM lane quarter) takes the query heads h of
-    // the column group with h % 4 == e, so a head's columns never split across warps, and
-    // a quarter of the key's dimensions for |k|^2.  Groups 1-3 hand (sum of head maxima,
-    // |k|^2 share) to group 0 through a shared-memory slot, and group 0 adds them in group
-    // order and writes the pooled score.  Four warps per SM sub-partition interleave
-    // their TMEM loads, which a single warp cannot overlap with its own arithmetic.
+    // the column group with h % 4 == e, so a head's columns never leave the thread that
+    // owns the key, and a quarter of the key's dimensions for |k|^2.  Every group hands
+    // (sum of head maxima, |k|^2 share) to a shared-memory slot; the tile's merging group
+    // adds the four in group order one tile later and writes the pooled score.
+    // Four warps per SM sub-partition interleave their TMEM loads, which a single warp
+    // cannot overlap with its own arithmetic.
     const int e = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
@@ -243,9 +266,30 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     int stage = 0, cur = -1, nsl_done = 0, ncols = 0, nmerge = 0;
     uint32_t kph = 0;
     bool ok = true;
+    int b, g, cg, tile, tiles;
+    stc_decode(p, tab, u_lo, b, g, cg, tile);
+    tiles = (tab.prefix[b] + STC_BM - 1) / STC_BM;
+    int pb = 0, pg = 0, pcg = 0, ptile = 0;
+    auto merge_tile = [&](int m, int mb, int mg, int mcg, int mtile) -> bool {
+      const int slot = m & 1;
+      const uint32_t mph = (uint32_t)(m >> 1) & 1u;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_sleep(&mfull[slot], mph))) return false;
+      float2 o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) o[q] = mslot[(slot * 4 + q) * STC_BM + row];
+      ptx::mbar_arrive(&mempty[slot]);
+      const float msum = ((o[0].x + o[1].x) + o[2].x) + o[3].x;   // group order
+      const float mss = ((o[0].y + o[1].y) + o[2].y) + o[3].y;
+      const float knorm = sqrtf(mss);
+      const int j = mtile * STC_BM + row;
+      if (j < tab.prefix[mb]) {
+        const float sc = knorm > 0.f ? (p.ncg == 1 ? msum * p.inv_G : msum) / knorm : 0.f;
+        pooled[mcg * p.cg_stride + (size_t)(mb * p.h_kv + mg) * p.pooled_stride + j] = sc;
+      }
+      return true;
+    };
     for (int u = u_lo; u < u_hi && ok; ++u) {
-      int b, g, cg, tile;
-      stc_decode(p, tab, u, b, g, cg, tile);
+      if (u != u_lo) stc_next(p, tab, b, g, cg, tile, tiles);
       const int key3 = (b * p.h_kv + g) * p.ncg + cg;
       if (key3 != cur) {
         ptx::named_bar(1, 32 * STC_EPI_WARPS);
@@ -273,7 +317,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       // slot this warp never waited for could otherwise count toward the slot's previous
       // use.  Then |k|^2 over this group's dimensions from the swizzled tile.
       for (int kb = 0; kb < KB; ++kb)
-        if (ok) ok = ptx::mbar_wait(&kfull[st[kb]], sph[kb]);
+        if (ok) ok = ptx::mbar_wait_sleep(&kfull[st[kb]], sph[kb]);
       float ss = 0.f;
       if (ok) {
         const uint8_t* rp = sK + st[kb_e] * Cfg::STAGE_BYTES + row * 128;
@@ -295,89 +339,83 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       if (!ok) break;
 
       // sum over this group's heads of max over the head's kept queries of s / |q| (+ bias)
+      auto range_max = [&](uint32_t tcol, int cbase, int ncol) -> float {
+        const float* ci = cpi + cbase;
+        const float* cb = cpb + cbase;
+        float run = -INFINITY;
+        for (int c = 0; c < ncol; c += 32) {
+          const int w = min(32, ncol - c);         // 32 or (odd tail) 16 columns
+          uint32_t r[32];
+          if (w == 32) ptx::tmem_ld32(lane_base + tcol + (uint32_t)c, r);
+          else ptx::tmem_ld16(lane_base + tcol + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(r));
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            if (q * 16 < w) {
+              float v[16];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 sc = reinterpret_cast<const float4*>(ci + c + q * 16)[i];
+                const uint32_t* rr = &r[q * 16 + 4 * i];
+                const float2 s01 = make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1]));
+                const float2 s23 = make_float2(__uint_as_float(rr[2]), __uint_as_float(rr[3]));
+                float2 v01, v23;
+                if (p.padded) {
+                  const float4 bi = reinterpret_cast<const float4*>(cb + c + q * 16)[i];
+                  v01 = ptx::fma2(s01, make_float2(sc.x, sc.y), make_float2(bi.x, bi.y));
+                  v23 = ptx::fma2(s23, make_float2(sc.z, sc.w), make_float2(bi.z, bi.w));
+                } else {
+                  v01 = ptx::mul2(s01, make_float2(sc.x, sc.y));
+                  v23 = ptx::mul2(s23, make_float2(sc.z, sc.w));
+                }
+                v[4 * i] = v01.x; v[4 * i + 1] = v01.y; v[4 * i + 2] = v23.x; v[4 * i + 3] = v23.y;
+              }
+              const float a0 = ptx::max3(v[0], v[1], v[2]), a1 = ptx::max3(v[3], v[4], v[5]);
+              const float a2 = ptx::max3(v[6], v[7], v[8]), a3 = ptx::max3(v[9], v[10], v[11]);
+              const float a4 = ptx::max3(v[12], v[13], v[14]);
+              run = ptx::max3(run, ptx::max3(a0, a1, a2), ptx::max3(a3, a4, v[15]));
+            }
+          }
+        }
+        return run;
+      };
       float sum = 0.f;
       for (int sl = 0; sl < nsl && ok; ++sl, ++nsl_done) {
         const int buf = nsl_done & 1;
         const uint32_t bph = (uint32_t)(nsl_done >> 1) & 1u;
         // every group waits for every slice before releasing it, which keeps the
         // accumulator's release barrier in step with its uses
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&accfull[buf], bph));
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&accfull[buf], bph));
         if (!ok) break;
         ptx::tc_fence_after();
+        // this group's whole heads h % 4 == e that the slice holds, in head order
         const int h_lo = sl == 0 ? 0 : hs0, h_hi = sl == 0 ? hs0 : nh;
-        for (int h = h_lo + ((e - h_lo) & 3); h < h_hi; h += 4) {
-          const uint32_t tcol = (uint32_t)(buf * STC_SLICE + (h - h_lo) * p.nkp);
-          const float* ci = cpi + h * p.nkp;
-          const float* cb = cpb + h * p.nkp;
-          float run = -INFINITY;
-          for (int c = 0; c < p.nkp; c += 32) {
-            const int w = min(32, p.nkp - c);       // 32 or (odd tail) 16 columns
-            uint32_t r[32];
-            if (w == 32) ptx::tmem_ld32(lane_base + tcol + (uint32_t)c, r);
-            else ptx::tmem_ld16(lane_base + tcol + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(r));
-            ptx::tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              if (q * 16 < w) {
-                float v[16];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float4 sc = reinterpret_cast<const float4*>(ci + c + q * 16)[i];
-                  const uint32_t* rr = &r[q * 16 + 4 * i];
-                  const float2 s01 = make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1]));
-                  const float2 s23 = make_float2(__uint_as_float(rr[2]), __uint_as_float(rr[3]));
-                  float2 v01, v23;
-                  if (p.padded) {
-                    const float4 bi = reinterpret_cast<const float4*>(cb + c + q * 16)[i];
-                    v01 = ptx::fma2(s01, make_float2(sc.x, sc.y), make_float2(bi.x, bi.y));
-                    v23 = ptx::fma2(s23, make_float2(sc.z, sc.w), make_float2(bi.z, bi.w));
-                  } else {
-                    v01 = ptx::mul2(s01, make_float2(sc.x, sc.y));
-                    v23 = ptx::mul2(s23, make_float2(sc.z, sc.w));
-                  }
-                  v[4 * i] = v01.x; v[4 * i + 1] = v01.y; v[4 * i + 2] = v23.x; v[4 * i + 3] = v23.y;
-                }
-                const float a0 = ptx::max3(v[0], v[1], v[2]), a1 = ptx::max3(v[3], v[4], v[5]);
-                const float a2 = ptx::max3(v[6], v[7], v[8]), a3 = ptx::max3(v[9], v[10], v[11]);
-                const float a4 = ptx::max3(v[12], v[13], v[14]);
-                run = ptx::max3(run, ptx::max3(a0, a1, a2), ptx::max3(a3, a4, v[15]));
-              }
-            }
-          }
-          sum += run;
-        }
+        for (int h = h_lo + ((e - h_lo) & 3); h < h_hi; h += 4)
+          sum += range_max((uint32_t)(buf * STC_SLICE + (h - h_lo) * p.nkp), h * p.nkp, p.nkp);
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&accempty[buf]);
       }
       if (!ok) break;
 
-      const int slot = nmerge & 1;
-      const uint32_t mph = (uint32_t)(nmerge >> 1) & 1u;
-      ++nmerge;
-      if (e != 0) {                                // hand this group's partials to group 0
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&mempty[slot], mph ^ 1u));
+      // Hand this tile's partials over, then merge the previous tile, whose partials are
+      // all in by now: the merging group rotates, and no group waits for the slowest one.
+      {
+        const int slot = nmerge & 1;
+        const uint32_t mph = (uint32_t)(nmerge >> 1) & 1u;
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&mempty[slot], mph ^ 1u));
         if (!ok) break;
-        mslot[(slot * 3 + (e - 1)) * STC_BM + row] = make_float2(sum, ss);
+        mslot[(slot * 4 + e) * STC_BM + row] = make_float2(sum, ss);
         ptx::mbar_arrive(&mfull[slot]);
-        continue;
       }
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&mfull[slot], mph));
-      if (!ok) break;
-#pragma unroll
-      for (int q = 0; q < 3; ++q) {
-        const float2 o = mslot[(slot * 3 + q) * STC_BM + row];
-        sum += o.x;
-        ss += o.y;
+      if (nmerge > 0 && e == ((nmerge - 1) & 3)) {
+        ok = merge_tile(nmerge - 1, pb, pg, pcg, ptile);
+        if (!ok) break;
       }
-      ptx::mbar_arrive(&mempty[slot]);
-      const float knorm = sqrtf(ss);
-      const int j = tile * STC_BM + row;
-      if (j < tab.prefix[b]) {
-        const float sc = knorm > 0.f ? (p.ncg == 1 ? sum * p.inv_G : sum) / knorm : 0.f;
-        pooled[cg * p.cg_stride + (size_t)(b * p.h_kv + g) * p.pooled_stride + j] = sc;
-      }
+      pb = b; pg = g; pcg = cg; ptile = tile;
+      ++nmerge;
     }
+    if (ok && nmerge > 0 && e == ((nmerge - 1) & 3)) merge_tile(nmerge - 1, pb, pg, pcg, ptile);
   }
 
   ptx::tc_fence_before();
