@@ -150,13 +150,13 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     if (lane == 0) {
       bool ok = true;
       if (rank == 1) {                     // tell CTA 0 that this CTA's query tile landed
-        ok = ptx::mbar_wait(qfull, 0);
+        ok = ptx::mbar_wait_sleep(qfull, 0);
         if (ok) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(qpeer), 0));
       }
       for (int j = 0; j < nblk && ok; ++j) {
         const int st = j % AT2_ST;
         const int row = kc_row0 + j * 128;
-        ok = ptx::mbar_wait(&kvempty[st], ((uint32_t)(j / AT2_ST) & 1u) ^ 1u);
+        ok = ptx::mbar_wait_sleep(&kvempty[st], ((uint32_t)(j / AT2_ST) & 1u) ^ 1u);
         if (!ok) break;
         if (rank == 0) ptx::mbar_expect_tx(&kvfull[st], 2u * (Cfg::KH_BYTES + Cfg::VH_BYTES));
         const uint32_t fbar = ptx::mapa_shared(ptx::smem_u32(&kvfull[st]), 0);
@@ -191,9 +191,9 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
                                   b0 + (uint32_t)(kb * 512 + k * 2), k_hi, idesc_s, (kb | k) ? 1u : 0u);
       };
       auto kv_landed = [&](int j) -> bool {
-        return ptx::mbar_wait_cluster(&kvfull[j % AT2_ST], (uint32_t)(j / AT2_ST) & 1u);
+        return ptx::mbar_wait_cluster_sleep(&kvfull[j % AT2_ST], (uint32_t)(j / AT2_ST) & 1u);
       };
-      bool ok = ptx::mbar_wait(qfull, 0) && ptx::mbar_wait_cluster(qpeer, 0);
+      bool ok = ptx::mbar_wait_sleep(qfull, 0) && ptx::mbar_wait_cluster_sleep(qpeer, 0);
       for (int j = 0; j < 2 && j < nblk && ok; ++j) {
         ok = kv_landed(j);
         if (!ok) break;
@@ -209,7 +209,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         const int st = j % AT2_ST;
         const bool more = j + 2 < nblk;
         if (more) ok = kv_landed(j + 2);
-        if (ok) ok = ptx::mbar_wait_cluster(&pready[j & 1], (uint32_t)(j >> 1) & 1u);
+        if (ok) ok = ptx::mbar_wait_cluster_sleep(&pready[j & 1], (uint32_t)(j >> 1) & 1u);
         if (!ok) break;
         ptx::tc_fence_after();
         // O += P(j) V(j); P(j) lies in buffer j % 2: keys 0-63 in columns 0-31, keys
@@ -262,7 +262,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     // after a failed (timed-out) wait a warp skips the work but keeps the exchanges.
     for (int j = 0; j < nblk; ++j) {
       const int buf = j & 1;
-      if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&sfull[buf], (uint32_t)(j >> 1) & 1u));
+      if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&sfull[buf], (uint32_t)(j >> 1) & 1u));
       if (!ok) {
         (void)exchange(0.f, true);
         continue;
@@ -330,7 +330,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         // released.  The parity wait is unambiguous: the stage's previous release,
         // P.V(j-1-ST), precedes S(j) (which was issued after P.V(j-2)), and its next one,
         // P.V(j-1+ST), needs this warp's P of a later block
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&kvempty[(j - 1) % AT2_ST], (uint32_t)((j - 1) / AT2_ST) & 1u));
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&kvempty[(j - 1) % AT2_ST], (uint32_t)((j - 1) / AT2_ST) & 1u));
         if (ok) ptx::tc_fence_after();
 #pragma unroll
         for (int c = 0; c < (ok ? DH : 0); c += 16) {
@@ -352,7 +352,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     }
     // epilogue: O / l -> bf16 rows of out[b, g*G + hl, t, :], this half's columns, once
     // the last P.V has released its stage (its commit covers every earlier MMA)
-    if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&kvempty[(nblk - 1) % AT2_ST], (uint32_t)((nblk - 1) / AT2_ST) & 1u));
+    if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&kvempty[(nblk - 1) % AT2_ST], (uint32_t)((nblk - 1) / AT2_ST) & 1u));
     const float l_row = exchange(ok ? l_run : 0.f, false);   // every pair member reaches this
     if (ok) {
       ptx::tc_fence_after();

@@ -15,8 +15,11 @@
 //                      decision.  The same reads give, per pass, how many keys of lower-
 //                      ranked CTAs fall in bins better than the chosen digit; summed over the
 //                      passes that is this CTA's output offset, so emitting needs no further
-//                      exchange.  Ends with a cluster barrier arrive after its last remote
-//                      read: the caller waits (cluster_wait) before it exits.
+//                      exchange.  The passes stop early once the chosen bin holds exactly the
+//                      keys still to be selected: every key of that bin is selected, so the
+//                      bits below cannot matter (keys are then compared under the mask of
+//                      the bits fixed so far).  Ends with a cluster barrier arrive after its
+//                      last remote read: the caller waits (cluster_wait) before it exits.
 //   block_threshold    all n keys in this CTA's shared memory: the same passes with one
 //                      block barrier each (three histogram buffers, so clearing the next one
 //                      never races a slow warp's decision).
@@ -38,10 +41,12 @@ struct SelectSmem {
   int wcnt[2][32];                // per warp: keys better than / equal to the threshold
 };
 
-// The k-th best key thr and this CTA's share of the selection: the selected keys are those
-// better than thr and, in index order, the first eq_left of this CTA's keys equal to thr.
+// The k-th best key thr and this CTA's share of the selection: with keys compared under
+// mask (the bits the radix passes fixed), the selected keys are those better than thr and,
+// in index order, the first eq_left of this CTA's keys equal to thr.
 struct SelectThreshold {
   uint32_t thr;
+  uint32_t mask;
   int sel_before;                 // selected keys before this CTA's range
   int eq_left;
 };
@@ -74,10 +79,11 @@ __device__ __forceinline__ void load_bins8(const int* tab, int lane, int (&c)[8]
 
 // One warp's digit decision for the k-th best key from per-bin totals (and, when bef is
 // given, per-bin counts of lower-ranked CTAs).  Every lane returns the digit, the number of
-// keys in better bins (run) and, from bef, the lower ranks' keys in better bins (bb).
+// keys in better bins (run), the chosen bin's count and, from bef, the lower ranks' keys in
+// better bins (bb).
 template <bool BEST_IS_LARGEST, bool WITH_BEF>
 __device__ __forceinline__ void decide_digit(const int* tots, const int* bef, int k, int* digit,
-                                             int* run_out, int* bb_out) {
+                                             int* run_out, int* cnt_out, int* bb_out) {
   const int lane = threadIdx.x & 31;
   int c[8], e[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   load_bins8<BEST_IS_LARGEST>(tots, lane, c);
@@ -98,10 +104,10 @@ __device__ __forceinline__ void decide_digit(const int* tots, const int* bef, in
   const unsigned owners = __ballot_sync(0xffffffffu, excl < k && k <= incl);
   if (owners == 0u && threadIdx.x == 0) flag_error(ERR_BAD_INDEX);   // counts inconsistent
   const int owner = owners ? __ffs(owners) - 1 : 31;
-  int run = excl, pick = 7, eb = 0;
+  int run = excl, pick = 7, eb = 0, cnt = 0;
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
-    if (run + c[q] >= k) { pick = q; break; }
+    if (run + c[q] >= k) { pick = q; cnt = c[q]; break; }
     run += c[q];
     eb += e[q];
   }
@@ -112,6 +118,7 @@ __device__ __forceinline__ void decide_digit(const int* tots, const int* bef, in
   }
   pick = __shfl_sync(0xffffffffu, pick, owner);
   *run_out = __shfl_sync(0xffffffffu, run, owner);
+  *cnt_out = __shfl_sync(0xffffffffu, cnt, owner);
   *bb_out = WITH_BEF ? bb : 0;
   const int pos = 8 * owner + pick;
   *digit = BEST_IS_LARGEST ? 255 - pos : pos;
@@ -148,17 +155,19 @@ __device__ SelectThreshold cluster_threshold(cg::cluster_group& cl, SelectSmem& 
       sm.hist[(pass + 1) & 1][tid] = 0;          // its remote readers passed the barrier above
     }
     __syncthreads();
-    int digit, run, bb;
-    decide_digit<BEST_IS_LARGEST, true>(sm.tots, sm.bef, k, &digit, &run, &bb);
+    int digit, run, cnt, bb;
+    decide_digit<BEST_IS_LARGEST, true>(sm.tots, sm.bef, k, &digit, &run, &cnt, &bb);
     better_before += bb;
-    if (pass == 3) eq_before = sm.bef[digit];
+    eq_before = sm.bef[digit];
     prefix |= (uint32_t)digit << shift;
     mask |= 0xFFu << shift;
     k -= run;
+    if (cnt == k) break;                         // the whole bin is selected
   }
   cluster_arrive();                              // last remote read done
   SelectThreshold t;
   t.thr = prefix;
+  t.mask = mask;
   t.sel_before = better_before + min(k, eq_before);
   t.eq_left = max(0, k - eq_before);
   return t;
@@ -182,14 +191,16 @@ __device__ SelectThreshold block_threshold(SelectSmem& sm, KeyFn key_at, int n, 
       if ((key & mask) == prefix) atomicAdd(&hcur[(key >> shift) & 255u], 1);
     }
     __syncthreads();
-    int digit, run, bb;
-    decide_digit<BEST_IS_LARGEST, false>(hcur, nullptr, k, &digit, &run, &bb);
+    int digit, run, cnt, bb;
+    decide_digit<BEST_IS_LARGEST, false>(hcur, nullptr, k, &digit, &run, &cnt, &bb);
     prefix |= (uint32_t)digit << shift;
     mask |= 0xFFu << shift;
     k -= run;
+    if (cnt == k) break;                         // the whole bin is selected
   }
   SelectThreshold t;
   t.thr = prefix;
+  t.mask = mask;
   t.sel_before = 0;
   t.eq_left = k;
   return t;
@@ -208,7 +219,7 @@ __device__ void ordered_emit(SelectSmem& sm, KeyFn key_at, int lo, int hi, const
   for (int base = wlo; base < whi; base += 32) {
     const int j = base + lane;
     const bool v = j < whi;
-    const uint32_t key = v ? key_at(j) : 0u;
+    const uint32_t key = v ? (key_at(j) & t.mask) : 0u;
     cb += __popc(__ballot_sync(0xffffffffu, v && better<BEST_IS_LARGEST>(key, t.thr)));
     ce += __popc(__ballot_sync(0xffffffffu, v && key == t.thr));
   }
@@ -229,7 +240,7 @@ __device__ void ordered_emit(SelectSmem& sm, KeyFn key_at, int lo, int hi, const
   for (int base = wlo; base < whi; base += 32) {
     const int j = base + lane;
     const bool v = j < whi;
-    const uint32_t key = v ? key_at(j) : 0u;
+    const uint32_t key = v ? (key_at(j) & t.mask) : 0u;
     const bool eq = v && key == t.thr;
     const unsigned meq = __ballot_sync(0xffffffffu, eq);
     const bool sel = (v && better<BEST_IS_LARGEST>(key, t.thr)) ||

@@ -31,6 +31,7 @@ constexpr int QSUB_WARPS = QSUB_THREADS / 32;
 constexpr int QSUB_MAX_ROWS = (QUOKA_MAX_CHUNK + QSUB_CS - 1) / QSUB_CS;
 constexpr int QSUB_LPR = 8;                   // lanes per query row
 constexpr int QSUB_RPS = 32 / QSUB_LPR;       // rows per warp step
+constexpr int QSUB_PULL = (QUOKA_MAX_CHUNK + QSUB_THREADS - 1) / QSUB_THREADS;   // keys pulled per thread
 
 // Per-lane view of a row: NV 16-byte vectors, vector v of lane l8 holding elements
 // [(8 v + l8) VE, (8 v + l8 + 1) VE).  U steps are in flight per warp (16 registers of
@@ -225,9 +226,18 @@ qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
     for (int t = lo + tid; t < hi; t += blockDim.x) emit(t, t);
   } else {
     cluster.sync();                            // every CTA's keys are final
-    for (int t = tid; t < C; t += blockDim.x) {
-      const int owner = t / S;
-      if (owner != rank) keys[t] = cluster.map_shared_rank(keys, owner)[t];
+    {                                          // all remote loads in flight before any store
+      uint32_t v[QSUB_PULL];
+#pragma unroll
+      for (int i = 0; i < QSUB_PULL; ++i) {
+        const int t = tid + i * QSUB_THREADS;
+        v[i] = (t < C && t / S != rank) ? cluster.map_shared_rank(keys, t / S)[t] : 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < QSUB_PULL; ++i) {
+        const int t = tid + i * QSUB_THREADS;
+        if (t < C && t / S != rank) keys[t] = v[i];
+      }
     }
     cluster_arrive();                          // remote reads of keys done; waited at the end
     __syncthreads();

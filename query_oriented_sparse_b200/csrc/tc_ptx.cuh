@@ -98,6 +98,30 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) 
     }
   }
 }
+// As mbar_try_wait_hint, with cluster-scope acquire.
+__device__ __forceinline__ bool mbar_try_wait_cluster_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+// As mbar_wait_sleep, with cluster-scope acquire.
+__device__ __forceinline__ bool mbar_wait_cluster_sleep(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    if (mbar_try_wait_cluster_hint(bar, parity, 1000000u)) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      flag_error(ERR_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
 // As mbar_wait, with cluster-scope acquire.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
