@@ -20,9 +20,10 @@
 // P(j) is written as bf16 into S buffer j % 2 and S(j+2) reuses that buffer after
 // P.V(j) has read it (one thread issues both, in order).
 //
-// In each CTA warp 0 loads and warps 2-9 run the softmax, one thread per query row and
-// 64-key half of the block (two warps per SM sub-partition share a row quarter); the
-// halves of a row agree on the block maximum through shared memory under a 64-thread
+// In each CTA warp 0 loads and warps 2-17 run the softmax, one thread per query row and
+// 32-key quarter of the block (four warps per SM sub-partition share a TMEM lane quarter,
+// so one warp's loads, exchanges and stores overlap the others' exponentials); the four
+// parts of a row agree on the block maximum through shared memory under a 128-thread
 // named barrier.  The online softmax keeps the running max per row in fp32 and rescales
 // O in TMEM only when it grows by more than 2^8.  Commits of the pair's MMAs arrive on
 // the barriers of both CTAs; the softmax warps of CTA 1 arrive on CTA 0's P-ready
@@ -35,7 +36,7 @@
 
 namespace quoka {
 
-constexpr int AT2_THREADS = 320;   // warp 0 load, warp 1 MMA (CTA 0), warps 2-9 softmax
+constexpr int AT2_THREADS = 576;   // warp 0 load, warp 1 MMA (CTA 0), warps 2-17 softmax
 constexpr int AT2_ST = 4;          // stages of (K half-tile, V half-tile) per block
 constexpr float AT2_RESCALE_LOG2 = 8.0f;
 
@@ -48,7 +49,7 @@ struct At2Cfg {
   static constexpr int V_BYTES = AT2_ST * VH_BYTES;
   // qfull, qpeer, stage full/empty ring, sfull[2], pready[2]
   static constexpr int NBAR = 2 + 2 * AT2_ST + 2 + 2;
-  static constexpr int XBUF = 128 * 4;
+  static constexpr int XBUF = 2 * 4 * 128 * 4;   // [phase][part][row] exchange slots
   static constexpr int SMEM = 1024 + Q_BYTES + K_BYTES + V_BYTES + NBAR * 8 + 16 + XBUF;
 };
 
@@ -86,7 +87,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
   uint64_t* kvfull = bars + 2;
   uint64_t* kvempty = kvfull + AT2_ST;
   uint64_t* sfull = kvempty + AT2_ST;      // [buffer], both CTAs
-  uint64_t* pready = sfull + 2;            // [buffer], CTA 0: 16 warps of the pair
+  uint64_t* pready = sfull + 2;            // [buffer], CTA 0: 32 softmax warps of the pair
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pready + 2);
   float* xbuf = reinterpret_cast<float*>(tmem_slot + 4);
 
@@ -109,7 +110,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     for (int s = 0; s < AT2_ST; ++s) { ptx::mbar_init(&kvfull[s], 1); ptx::mbar_init(&kvempty[s], 1); }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sfull[i], 1);
-      ptx::mbar_init(&pready[i], 16);
+      ptx::mbar_init(&pready[i], 32);
     }
     ptx::fence_mbar_init();
   }
@@ -212,13 +213,13 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         if (ok) ok = ptx::mbar_wait_cluster_sleep(&pready[j & 1], (uint32_t)(j >> 1) & 1u);
         if (!ok) break;
         ptx::tc_fence_after();
-        // O += P(j) V(j); P(j) lies in buffer j % 2: keys 0-63 in columns 0-31, keys
-        // 64-127 in columns 96-127
+        // O += P(j) V(j); P(j) lies in buffer j % 2: keys 32q .. 32q+31 in columns
+        // 32q .. 32q+15 (written by softmax part q)
         const uint32_t b0 = v_lo + (uint32_t)(st * (Cfg::VH_BYTES >> 4));
         const uint32_t pa = tmem + (uint32_t)((j & 1) * 128);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          ptx::mma_bf16_ts_pair(tmem + 256u, pa + (uint32_t)(k < 4 ? k * 8 : 96 + (k - 4) * 8),
+          ptx::mma_bf16_ts_pair(tmem + 256u, pa + (uint32_t)((k >> 1) * 32 + (k & 1) * 8),
                                 b0 + (uint32_t)(k * 128), v_hi, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
         if (more) {
           s_mmas(j + 2);
@@ -228,28 +229,25 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       }
     }
   } else {
-    // ---------------- softmax: warps 2-9, one row per thread and key half ----------------
-    const int half = ((warp - 2) >> 2) & 1;
+    // ---------------- softmax: warps 2-17, one row per thread and key quarter ----------------
+    const int part = ((warp - 2) >> 2) & 3;                 // key quarter of each block
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                      // row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    constexpr int DH = D / 2;
-    const uint32_t o_addr = tmem + lane_off + 256u + (uint32_t)(half * DH);
-    float* xslot = xbuf + r;
+    constexpr int DP = D / 4;                               // O columns of this part
+    const uint32_t o_addr = tmem + lane_off + 256u + (uint32_t)(part * DP);
     const int bar_id = 1 + quarter;
     const uint32_t pready_c0 = ptx::mapa_shared(ptx::smem_u32(pready), 0);   // CTA 0's pready[0]
-    // half 0 posts v, half 1 combines it with its own and posts the result for half 0
+    // the four parts of a row post their values and each combines all four in part order;
+    // slots alternate between two sets, so one barrier per exchange suffices
+    int xphase = 0;
     auto exchange = [&](float v, bool is_max) -> float {
-      if (half == 0) *xslot = v;
-      ptx::named_bar(bar_id, 64);
-      float res = v;
-      if (half == 1) {
-        res = is_max ? fmaxf(v, *xslot) : v + *xslot;
-        *xslot = res;
-      }
-      ptx::named_bar(bar_id, 64);
-      if (half == 0) res = *xslot;
-      return res;
+      float* slot = xbuf + (xphase & 1) * 512 + r;
+      slot[part * 128] = v;
+      ptx::named_bar(bar_id, 128);
+      const float a0 = slot[0], a1 = slot[128], a2 = slot[256], a3 = slot[384];
+      ++xphase;
+      return is_max ? fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) : (a0 + a1) + (a2 + a3);
     };
     const int hl = r / p.TP;
     const int t = t0 + (int)rank * p.TP + r % p.TP;
@@ -257,8 +255,8 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     const int tmin = t0 + (int)rank * p.TP;                 // smallest position in this tile
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    // Both warps of a row pair take part in exactly one exchange per block and one at
-    // the end, whatever happens, so the named barrier never waits for a warp that left:
+    // The four warps of a row quarter take part in exactly one exchange per block and one
+    // at the end, whatever happens, so the named barrier never waits for a warp that left:
     // after a failed (timed-out) wait a warp skips the work but keeps the exchanges.
     for (int j = 0; j < nblk; ++j) {
       const int buf = j & 1;
@@ -268,21 +266,21 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         continue;
       }
       ptx::tc_fence_after();
-      const uint32_t s_addr = tmem + lane_off + (uint32_t)(buf * 128 + half * 64);
-      const uint32_t p_addr = tmem + lane_off + (uint32_t)(buf * 128 + half * 96);
-      float s[64];
-#pragma unroll
-      for (int c = 0; c < 64; c += 32) {
+      // this part's 32 keys of S(j); P(j) goes to the first 16 columns of the same place
+      const uint32_t s_addr = tmem + lane_off + (uint32_t)(buf * 128 + part * 32);
+      const uint32_t p_addr = s_addr;
+      float s[32];
+      {
         uint32_t u[32];
-        ptx::tmem_ld32(s_addr + (uint32_t)c, u);
+        ptx::tmem_ld32(s_addr, u);
+        ptx::tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(u[i]);
+        for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(u[i]);
       }
-      ptx::tmem_ld_wait();
-      const int kb0 = j * 128 + half * 64;
-      if (kb0 + 63 >= nsel + tmin || kb0 + 63 >= nkeys) {   // keys reach the causal part
+      const int kb0 = j * 128 + part * 32;
+      if (kb0 + 31 >= nsel + tmin || kb0 + 31 >= nkeys) {   // keys reach the causal part
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < 32; ++c) {
           const int kk = kb0 + c;
           const bool valid = kk < nkeys && (kk < nsel || kk - nsel <= t);
           if (!valid) s[c] = -INFINITY;
@@ -292,14 +290,14 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       {
         float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-        for (int c = 4; c < 60; c += 8) {
+        for (int c = 4; c < 28; c += 8) {
           m0 = ptx::max3(m0, s[c], s[c + 1]);
           m1 = ptx::max3(m1, s[c + 2], s[c + 3]);
           m2 = ptx::max3(m2, s[c + 4], s[c + 5]);
           m3 = ptx::max3(m3, s[c + 6], s[c + 7]);
         }
-        m0 = ptx::max3(m0, s[60], s[61]);
-        m1 = ptx::max3(m1, s[62], s[63]);
+        m0 = ptx::max3(m0, s[28], s[29]);
+        m1 = ptx::max3(m1, s[30], s[31]);
         mx = exchange(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), true);
       }
       const float m_cand = mx * p.scale_log2;
@@ -312,17 +310,16 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 64; c += 32) {
+      {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ptx::ex2_approx(fmaf(s[c + 2 * i], p.scale_log2, -m_use));
-          const float p1 = ptx::ex2_approx(fmaf(s[c + 2 * i + 1], p.scale_log2, -m_use));
+          const float p0 = ptx::ex2_approx(fmaf(s[2 * i], p.scale_log2, -m_use));
+          const float p1 = ptx::ex2_approx(fmaf(s[2 * i + 1], p.scale_log2, -m_use));
           ls[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        ptx::tmem_st16(p_addr + (uint32_t)(c / 2), pk);
+        ptx::tmem_st16(p_addr, pk);
       }
       l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
@@ -333,7 +330,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&kvempty[(j - 1) % AT2_ST], (uint32_t)((j - 1) / AT2_ST) & 1u));
         if (ok) ptx::tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < (ok ? DH : 0); c += 16) {
+        for (int c = 0; c < (ok ? DP : 0); c += 16) {
           uint32_t u[16];
           ptx::tmem_ld16(o_addr + (uint32_t)c, u);
           ptx::tmem_ld_wait();
@@ -350,7 +347,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       // would stall the warp on its unrelated outstanding memory operations
       if (ok && lane == 0) ptx::mbar_arrive_cluster_relaxed(pready_c0 + (uint32_t)(buf * 8));
     }
-    // epilogue: O / l -> bf16 rows of out[b, g*G + hl, t, :], this half's columns, once
+    // epilogue: O / l -> bf16 rows of out[b, g*G + hl, t, :], this part's columns, once
     // the last P.V has released its stage (its commit covers every earlier MMA)
     if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&kvempty[(nblk - 1) % AT2_ST], (uint32_t)((nblk - 1) / AT2_ST) & 1u));
     const float l_row = exchange(ok ? l_run : 0.f, false);   // every pair member reaches this
@@ -358,9 +355,9 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       ptx::tc_fence_after();
       const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
       __nv_bfloat16* orow = out + ((size_t)(b * p.h_q + g * p.G + (row_valid ? hl : 0)) * p.C +
-                                   (row_valid ? t : 0)) * D + half * DH;
+                                   (row_valid ? t : 0)) * D + part * DP;
 #pragma unroll
-      for (int c = 0; c < DH; c += 16) {
+      for (int c = 0; c < DP; c += 16) {
         uint32_t u[16];
         ptx::tmem_ld16(o_addr + (uint32_t)c, u);
         ptx::tmem_ld_wait();
