@@ -13,19 +13,24 @@
 //               split by columns, CTA r holding columns 64r .. 64r+63.
 // So each SM loads half of every K and V tile (tiled TMA, 128-byte swizzle, bytes
 // counted on CTA 0's barrier) and still feeds 256 query rows per tile pair, and each
-// SM's TMEM holds only its own tile: S in two 128-column buffers and O (384 of 512
-// columns).  With S double-buffered the tensor cores compute S(j+1) while the softmax
-// works on S(j):
+// SM's TMEM holds only its own tile: S in two 128-column buffers and two O accumulators
+// (512 columns).  The key blocks are split by parity between two softmax groups, each
+// with its own running max, row sum and O (a split of the key range, combined at the
+// end like a split-K reduction):
 //   MMA order   S(0) S(1) | P.V(0) S(2) | P.V(1) S(3) | ...   (P.V(j) waits for P(j))
+//   P.V(j) accumulates into O_{j % 2}
 // P(j) is written as bf16 into S buffer j % 2 and S(j+2) reuses that buffer after
 // P.V(j) has read it (one thread issues both, in order).
 //
-// In each CTA warp 0 loads and warps 2-17 run the softmax, one thread per query row and
-// 32-key quarter of the block (four warps per SM sub-partition share a TMEM lane quarter,
-// so one warp's loads, exchanges and stores overlap the others' exponentials); the four
-// parts of a row agree on the block maximum through shared memory under a 128-thread
+// In each CTA warp 0 loads and warps 2-17 run the softmax: warps 2-9 take the even key
+// blocks and warps 10-17 the odd ones, one thread per query row and 64-key half of a
+// block.  Each SM sub-partition holds two warps of each group, a block apart, so one
+// group's exponentials overlap the other group's TMEM loads, exchange and waits.  The
+// halves of a row agree on the block maximum through shared memory under a 64-thread
 // named barrier.  The online softmax keeps the running max per row in fp32 and rescales
-// O in TMEM only when it grows by more than 2^8.  Commits of the pair's MMAs arrive on
+// its group's O in TMEM only when the max grows by more than 2^8; at the end the two
+// groups meet per row quarter and write O = (O_0 f_0 + O_1 f_1) / (l_0 f_0 + l_1 f_1),
+// f_g = 2^(m_g - max(m_0, m_1)).  Commits of the pair's MMAs arrive on
 // the barriers of both CTAs; the softmax warps of CTA 1 arrive on CTA 0's P-ready
 // barrier through its cluster address.  Every mbarrier wait is bounded; the only
 // unbounded waits are the two cluster barriers, which every thread of both CTAs reaches
@@ -49,7 +54,7 @@ struct At2Cfg {
   static constexpr int V_BYTES = AT2_ST * VH_BYTES;
   // qfull, qpeer, stage full/empty ring, sfull[2], pready[2]
   static constexpr int NBAR = 2 + 2 * AT2_ST + 2 + 2;
-  static constexpr int XBUF = 2 * 4 * 128 * 4;   // [phase][part][row] exchange slots
+  static constexpr int XBUF = (2 * 2 * 2 * 128 + 2 * 2 * 128) * 4;   // exchange slots, then (m, l) per group
   static constexpr int SMEM = 1024 + Q_BYTES + K_BYTES + V_BYTES + NBAR * 8 + 16 + XBUF;
 };
 
@@ -87,7 +92,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
   uint64_t* kvfull = bars + 2;
   uint64_t* kvempty = kvfull + AT2_ST;
   uint64_t* sfull = kvempty + AT2_ST;      // [buffer], both CTAs
-  uint64_t* pready = sfull + 2;            // [buffer], CTA 0: 32 softmax warps of the pair
+  uint64_t* pready = sfull + 2;            // [buffer], CTA 0: the 16 warps of one group of the pair
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pready + 2);
   float* xbuf = reinterpret_cast<float*>(tmem_slot + 4);
 
@@ -110,7 +115,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     for (int s = 0; s < AT2_ST; ++s) { ptx::mbar_init(&kvfull[s], 1); ptx::mbar_init(&kvempty[s], 1); }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sfull[i], 1);
-      ptx::mbar_init(&pready[i], 32);
+      ptx::mbar_init(&pready[i], 16);
     }
     ptx::fence_mbar_init();
   }
@@ -213,14 +218,14 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         if (ok) ok = ptx::mbar_wait_cluster_sleep(&pready[j & 1], (uint32_t)(j >> 1) & 1u);
         if (!ok) break;
         ptx::tc_fence_after();
-        // O += P(j) V(j); P(j) lies in buffer j % 2: keys 32q .. 32q+31 in columns
-        // 32q .. 32q+15 (written by softmax part q)
+        // O_{j%2} += P(j) V(j); P(j) lies in buffer j % 2: keys 0-63 in columns 0-31, keys
+        // 64-127 in columns 96-127
         const uint32_t b0 = v_lo + (uint32_t)(st * (Cfg::VH_BYTES >> 4));
         const uint32_t pa = tmem + (uint32_t)((j & 1) * 128);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          ptx::mma_bf16_ts_pair(tmem + 256u, pa + (uint32_t)((k >> 1) * 32 + (k & 1) * 8),
-                                b0 + (uint32_t)(k * 128), v_hi, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+          ptx::mma_bf16_ts_pair(tmem + 256u + (uint32_t)((j & 1) * 128), pa + (uint32_t)(k < 4 ? k * 8 : 96 + (k - 4) * 8),
+                                b0 + (uint32_t)(k * 128), v_hi, idesc_o, (j > 1 || k > 0) ? 1u : 0u);
         if (more) {
           s_mmas(j + 2);
           ptx::tc_commit_pair(&sfull[j & 1], kBoth);
@@ -229,25 +234,26 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       }
     }
   } else {
-    // ---------------- softmax: warps 2-17, one row per thread and key quarter ----------------
-    const int part = ((warp - 2) >> 2) & 3;                 // key quarter of each block
+    // ---------------- softmax: warps 2-17 in two groups over even / odd key blocks ----------------
+    const int grp = ((warp - 2) >> 3) & 1;                  // 0: even blocks, 1: odd blocks
+    const int half = ((warp - 2) >> 2) & 1;                 // key half of each block
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                      // row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    constexpr int DP = D / 4;                               // O columns of this part
-    const uint32_t o_addr = tmem + lane_off + 256u + (uint32_t)(part * DP);
-    const int bar_id = 1 + quarter;
+    constexpr int DH = D / 2;
+    const uint32_t o_addr = tmem + lane_off + 256u + (uint32_t)(grp * 128 + half * DH);
+    const int bar_id = 1 + grp * 4 + quarter;
     const uint32_t pready_c0 = ptx::mapa_shared(ptx::smem_u32(pready), 0);   // CTA 0's pready[0]
-    // the four parts of a row post their values and each combines all four in part order;
-    // slots alternate between two sets, so one barrier per exchange suffices
+    // the two halves of a row in a group post their values and each combines both; slots
+    // alternate between two sets, so one barrier per exchange suffices
     int xphase = 0;
     auto exchange = [&](float v, bool is_max) -> float {
-      float* slot = xbuf + (xphase & 1) * 512 + r;
-      slot[part * 128] = v;
-      ptx::named_bar(bar_id, 128);
-      const float a0 = slot[0], a1 = slot[128], a2 = slot[256], a3 = slot[384];
+      float* slot = xbuf + ((xphase & 1) * 2 + grp) * 256 + r;
+      slot[half * 128] = v;
+      ptx::named_bar(bar_id, 64);
+      const float a0 = slot[0], a1 = slot[128];
       ++xphase;
-      return is_max ? fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) : (a0 + a1) + (a2 + a3);
+      return is_max ? fmaxf(a0, a1) : a0 + a1;
     };
     const int hl = r / p.TP;
     const int t = t0 + (int)rank * p.TP + r % p.TP;
@@ -255,32 +261,35 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     const int tmin = t0 + (int)rank * p.TP;                 // smallest position in this tile
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    // The four warps of a row quarter take part in exactly one exchange per block and one
-    // at the end, whatever happens, so the named barrier never waits for a warp that left:
-    // after a failed (timed-out) wait a warp skips the work but keeps the exchanges.
-    for (int j = 0; j < nblk; ++j) {
-      const int buf = j & 1;
+    int jlast = -1;
+    // The two warps of a row quarter in a group take part in exactly one exchange per block
+    // of the group and one at the end, whatever happens, so the named barrier never waits
+    // for a warp that left: after a failed (timed-out) wait a warp skips the work but keeps
+    // the exchanges.
+    for (int j = grp; j < nblk; j += 2) {
+      const int buf = grp;                                  // == j % 2
+      jlast = j;
       if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&sfull[buf], (uint32_t)(j >> 1) & 1u));
       if (!ok) {
         (void)exchange(0.f, true);
         continue;
       }
       ptx::tc_fence_after();
-      // this part's 32 keys of S(j); P(j) goes to the first 16 columns of the same place
-      const uint32_t s_addr = tmem + lane_off + (uint32_t)(buf * 128 + part * 32);
-      const uint32_t p_addr = s_addr;
-      float s[32];
-      {
+      const uint32_t s_addr = tmem + lane_off + (uint32_t)(buf * 128 + half * 64);
+      const uint32_t p_addr = tmem + lane_off + (uint32_t)(buf * 128 + half * 96);
+      float s[64];
+#pragma unroll
+      for (int c = 0; c < 64; c += 32) {
         uint32_t u[32];
-        ptx::tmem_ld32(s_addr, u);
-        ptx::tmem_ld_wait();
+        ptx::tmem_ld32(s_addr + (uint32_t)c, u);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(u[i]);
+        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(u[i]);
       }
-      const int kb0 = j * 128 + part * 32;
-      if (kb0 + 31 >= nsel + tmin || kb0 + 31 >= nkeys) {   // keys reach the causal part
+      ptx::tmem_ld_wait();
+      const int kb0 = j * 128 + half * 64;
+      if (kb0 + 63 >= nsel + tmin || kb0 + 63 >= nkeys) {   // keys reach the causal part
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < 64; ++c) {
           const int kk = kb0 + c;
           const bool valid = kk < nkeys && (kk < nsel || kk - nsel <= t);
           if (!valid) s[c] = -INFINITY;
@@ -290,14 +299,14 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       {
         float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-        for (int c = 4; c < 28; c += 8) {
+        for (int c = 4; c < 60; c += 8) {
           m0 = ptx::max3(m0, s[c], s[c + 1]);
           m1 = ptx::max3(m1, s[c + 2], s[c + 3]);
           m2 = ptx::max3(m2, s[c + 4], s[c + 5]);
           m3 = ptx::max3(m3, s[c + 6], s[c + 7]);
         }
-        m0 = ptx::max3(m0, s[28], s[29]);
-        m1 = ptx::max3(m1, s[30], s[31]);
+        m0 = ptx::max3(m0, s[60], s[61]);
+        m1 = ptx::max3(m1, s[62], s[63]);
         mx = exchange(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), true);
       }
       const float m_cand = mx * p.scale_log2;
@@ -310,27 +319,29 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
-      {
+#pragma unroll
+      for (int c = 0; c < 64; c += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ptx::ex2_approx(fmaf(s[2 * i], p.scale_log2, -m_use));
-          const float p1 = ptx::ex2_approx(fmaf(s[2 * i + 1], p.scale_log2, -m_use));
+          const float p0 = ptx::ex2_approx(fmaf(s[c + 2 * i], p.scale_log2, -m_use));
+          const float p1 = ptx::ex2_approx(fmaf(s[c + 2 * i + 1], p.scale_log2, -m_use));
           ls[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        ptx::tmem_st16(p_addr, pk);
+        ptx::tmem_st16(p_addr + (uint32_t)(c / 2), pk);
       }
       l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // rescale O (blocks 0..j-1) once P.V(j-1) has finished, i.e. stage (j-1) % ST is
-        // released.  The parity wait is unambiguous: the stage's previous release,
-        // P.V(j-1-ST), precedes S(j) (which was issued after P.V(j-2)), and its next one,
-        // P.V(j-1+ST), needs this warp's P of a later block
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&kvempty[(j - 1) % AT2_ST], (uint32_t)((j - 1) / AT2_ST) & 1u));
+      if (j >= 2 && __any_sync(0xffffffffu, grow)) {
+        // rescale this group's O (blocks grp, grp + 2, ..., j - 2) once P.V(j-2) has
+        // finished, i.e. stage (j-2) % ST is released: S(j), which this warp has seen, was
+        // issued after P.V(j-2), so the wait does not stall.  The parity wait is
+        // unambiguous: the stage's next release, P.V(j-2+ST), needs this group's P of a
+        // later block
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&kvempty[(j - 2) % AT2_ST], (uint32_t)((j - 2) / AT2_ST) & 1u));
         if (ok) ptx::tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < (ok ? DP : 0); c += 16) {
+        for (int c = 0; c < (ok ? DH : 0); c += 16) {
           uint32_t u[16];
           ptx::tmem_ld16(o_addr + (uint32_t)c, u);
           ptx::tmem_ld_wait();
@@ -347,29 +358,47 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
       // would stall the warp on its unrelated outstanding memory operations
       if (ok && lane == 0) ptx::mbar_arrive_cluster_relaxed(pready_c0 + (uint32_t)(buf * 8));
     }
-    // epilogue: O / l -> bf16 rows of out[b, g*G + hl, t, :], this part's columns, once
-    // the last P.V has released its stage (its commit covers every earlier MMA)
-    if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&kvempty[(nblk - 1) % AT2_ST], (uint32_t)((nblk - 1) / AT2_ST) & 1u));
-    const float l_row = exchange(ok ? l_run : 0.f, false);   // every pair member reaches this
+    // epilogue: this group's O is final once its last P.V has released its stage (that
+    // commit covers every earlier MMA); the two groups then meet per row quarter and each
+    // thread writes 32 of the row's output columns from both groups' O:
+    //   out = (O_0 f_0 + O_1 f_1) / (l_0 f_0 + l_1 f_1),   f_g = 2^(m_g - max(m_0, m_1))
+    if (ok && jlast >= 0)
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&kvempty[jlast % AT2_ST], (uint32_t)(jlast / AT2_ST) & 1u));
+    const float l_grp = exchange(ok ? l_run : 0.f, false);   // every pair member reaches this
+    float* ml = xbuf + 2 * 2 * 2 * 128;                      // [m, l][group][row]
+    if (half == 0) {
+      ml[grp * 128 + r] = m_run;
+      ml[256 + grp * 128 + r] = ok ? l_grp : 0.f;
+    }
+    ptx::named_bar(9 + quarter, 128);                         // both groups of this row quarter
+    const float m0 = ml[r], m1 = ml[128 + r], l0 = ml[256 + r], l1 = ml[384 + r];
     if (ok) {
       ptx::tc_fence_after();
-      const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+      const float mm = fmaxf(m0, m1);
+      const float f0 = l0 > 0.f ? ptx::ex2_approx(m0 - mm) : 0.f;
+      const float f1 = l1 > 0.f ? ptx::ex2_approx(m1 - mm) : 0.f;
+      const float l = l0 * f0 + l1 * f1;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float g0 = f0 * inv_l, g1 = f1 * inv_l;
+      const int c0 = (grp * 2 + half) * 32;                   // this thread's output columns
       __nv_bfloat16* orow = out + ((size_t)(b * p.h_q + g * p.G + (row_valid ? hl : 0)) * p.C +
-                                   (row_valid ? t : 0)) * D + part * DP;
+                                   (row_valid ? t : 0)) * D + c0;
+      const uint32_t oa = tmem + lane_off + 256u + (uint32_t)c0;
 #pragma unroll
-      for (int c = 0; c < DP; c += 16) {
-        uint32_t u[16];
-        ptx::tmem_ld16(o_addr + (uint32_t)c, u);
+      for (int c = 0; c < 32; c += 16) {
+        uint32_t u0[16], u1[16];
+        ptx::tmem_ld16(oa + (uint32_t)c, u0);
+        ptx::tmem_ld16(oa + 128u + (uint32_t)c, u1);
         ptx::tmem_ld_wait();
+        float o[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          o[i] = (g0 > 0.f ? __uint_as_float(u0[i]) * g0 : 0.f) + (g1 > 0.f ? __uint_as_float(u1[i]) * g1 : 0.f);
         uint4 w0, w1;
-        w0.x = pack_bf16x2(__uint_as_float(u[0]) * inv_l, __uint_as_float(u[1]) * inv_l);
-        w0.y = pack_bf16x2(__uint_as_float(u[2]) * inv_l, __uint_as_float(u[3]) * inv_l);
-        w0.z = pack_bf16x2(__uint_as_float(u[4]) * inv_l, __uint_as_float(u[5]) * inv_l);
-        w0.w = pack_bf16x2(__uint_as_float(u[6]) * inv_l, __uint_as_float(u[7]) * inv_l);
-        w1.x = pack_bf16x2(__uint_as_float(u[8]) * inv_l, __uint_as_float(u[9]) * inv_l);
-        w1.y = pack_bf16x2(__uint_as_float(u[10]) * inv_l, __uint_as_float(u[11]) * inv_l);
-        w1.z = pack_bf16x2(__uint_as_float(u[12]) * inv_l, __uint_as_float(u[13]) * inv_l);
-        w1.w = pack_bf16x2(__uint_as_float(u[14]) * inv_l, __uint_as_float(u[15]) * inv_l);
+        w0.x = pack_bf16x2(o[0], o[1]);   w0.y = pack_bf16x2(o[2], o[3]);
+        w0.z = pack_bf16x2(o[4], o[5]);   w0.w = pack_bf16x2(o[6], o[7]);
+        w1.x = pack_bf16x2(o[8], o[9]);   w1.y = pack_bf16x2(o[10], o[11]);
+        w1.z = pack_bf16x2(o[12], o[13]); w1.w = pack_bf16x2(o[14], o[15]);
         if (row_valid) {
           reinterpret_cast<uint4*>(orow + c)[0] = w0;
           reinterpret_cast<uint4*>(orow + c)[1] = w1;

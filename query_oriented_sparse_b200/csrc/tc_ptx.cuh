@@ -86,9 +86,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
   }
 }
-// As mbar_wait, each try sleeping until the phase completes (or 1 ms passes).
+// As mbar_wait: a few plain tries first (a phase about to complete is seen without a
+// wake-up delay), then each try sleeps until the phase completes (or 1 ms passes).
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+  for (int i = 0; i < 16; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (;;) {
     if (mbar_try_wait_hint(bar, parity, 1000000u)) return true;
@@ -112,7 +114,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster_hint(uint64_t* bar, uint32
 }
 // As mbar_wait_sleep, with cluster-scope acquire.
 __device__ __forceinline__ bool mbar_wait_cluster_sleep(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+  for (int i = 0; i < 16; ++i)
+    if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (;;) {
     if (mbar_try_wait_cluster_hint(bar, parity, 1000000u)) return true;
