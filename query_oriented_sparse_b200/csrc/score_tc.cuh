@@ -383,18 +383,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       for (int sl = 0; sl < nsl && ok; ++sl, ++nsl_done) {
         const int buf = nsl_done & 1;
         const uint32_t bph = (uint32_t)(nsl_done >> 1) & 1u;
-        // every group waits for every slice before releasing it, which keeps the
-        // accumulator's release barrier in step with its uses
+        // only groups with heads in the slice wait for it; the first of them also releases
+        // it for the groups without any, so those move on at once
+        const int h_lo = sl == 0 ? 0 : hs0, h_hi = sl == 0 ? hs0 : nh;
+        const int h_first = h_lo + ((e - h_lo) & 3);
+        if (h_first >= h_hi) continue;
+        const int nidle = 4 - min(4, h_hi - h_lo);
         ok = __all_sync(0xffffffffu, ptx::mbar_wait_sleep(&accfull[buf], bph));
         if (!ok) break;
         ptx::tc_fence_after();
-        // this group's whole heads h % 4 == e that the slice holds, in head order
-        const int h_lo = sl == 0 ? 0 : hs0, h_hi = sl == 0 ? hs0 : nh;
-        for (int h = h_lo + ((e - h_lo) & 3); h < h_hi; h += 4)
+        for (int h = h_first; h < h_hi; h += 4)
           sum += range_max((uint32_t)(buf * STC_SLICE + (h - h_lo) * p.nkp), h * p.nkp, p.nkp);
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&accempty[buf]);
+        if (lane == 0) ptx::mbar_arrive_count(&accempty[buf], 1u + (e == (h_lo & 3) ? (uint32_t)nidle : 0u));
       }
       if (!ok) break;
 
