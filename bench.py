@@ -367,8 +367,9 @@ def run_ours(args, w):
                     t0.record(s_in)
                 qb[b].copy_(q_h, non_blocking=True)
                 for (a, b_), kh, vh in zip(kv_rows, kc_h, vc_h):
-                    kb[b][:, a:b_].copy_(kh, non_blocking=True)
-                    vb[b][:, a:b_].copy_(vh, non_blocking=True)
+                    for hh in range(kh.shape[0]):          # one contiguous copy per KV head
+                        kb[b][hh, a:b_].copy_(kh[hh], non_blocking=True)
+                        vb[b][hh, a:b_].copy_(vh[hh], non_blocking=True)
                 ev_in[b].record(s_in)
             stream.wait_event(ev_in[b])
             if i >= 2:
