@@ -1,6 +1,7 @@
 """Throughput of one chunked-prefill step (QUOKA selection + sparse chunk attention).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py --prefill [prompt_128k] [--steps K] [--warmup W]
 
 A step is one pass of the whole hot path over one batch of synthetic input: the
 select call (query subselect, cosine scoring + pooling, top-B) and the attention
@@ -9,6 +10,11 @@ chunk 4096, H_q 32, H_kv 8, d 128, Nq 128, B 16384, bf16).  Each timed step is
 bracketed by CUDA events on the launching stream, with a 256 MB L2 flush before it
 (outside the events).  Under torchrun every rank runs its own independent chunk step
 (weak scaling, no collective on the data path) and the slowest rank's time is used.
+
+`--prefill` instead times a whole prompt (33 chunks of the 128K-context shapes) through
+the prefill call, which appends each chunk's K/V to the cache, selects and attends: the
+attention path's time to first token, with a dense causal SDPA over the same prompt
+beside it for context.
 
 Rank 0 prints one JSON line.  `--impl reference` times the fp64 CPU oracle instead
 (test infrastructure, run on the host cores on a bounded sample of the workload).
@@ -439,6 +445,146 @@ def run_ours(args, w):
     return 0
 
 
+# --------------------------------------------------------------------------------------
+# whole-prompt prefill (time to first token of the attention path)
+# --------------------------------------------------------------------------------------
+
+PREFILL_METRIC = "whole-prompt chunked prefill, attention-path time to first token, 1 B200"
+
+
+def prompt_inputs(w, t, dev):
+    """Chunk-major prompt tensors on the device: q [n, batch, h_q, C, d] and the
+    prompt's own K/V rows k_new, v_new [n, batch, h_kv, C, d]."""
+    n, C, d = w.prompt_chunks, w.chunk, w.head_dim
+    q = t.q.view(w.batch, w.h_q, n, C, d).permute(2, 0, 1, 3, 4).contiguous().to(dev)
+
+    def rows(cache):
+        per_seq = [cache[:, t.kv_off[b]:t.kv_off[b] + n * C].reshape(w.h_kv, n, C, d)
+                   for b in range(w.batch)]
+        return torch.stack(per_seq, 0).permute(2, 0, 1, 3, 4).contiguous().to(dev)
+    return q, rows(t.k_cache), rows(t.v_cache)
+
+
+def prompt_stage_model(w):
+    """stage_model summed over the prompt's chunk steps."""
+    tot = None
+    for c, budget in enumerate(w.budgets_of_chunks()):
+        step = W.custom(h_q=w.h_q, h_kv=w.h_kv, head_dim=w.head_dim, chunk=w.chunk,
+                        prefix=tuple(p + c * w.chunk for p in w.prefix), nq=w.nq,
+                        budget=budget, dtype=w.dtype)
+        st = stage_model(step)
+        if c == 0 or budget == 0:                  # no selection runs on this chunk
+            for k in ("qsub", "score", "topk"):
+                st[k] = {"bytes": 0.0, "flops": 0.0}
+        if tot is None:
+            tot = st
+        else:
+            for k in tot:
+                for m in tot[k]:
+                    tot[k][m] += st[k][m]
+    return tot
+
+
+def dense_reference_ms(q, k_new, v_new, steps, flush):
+    """Dense causal attention over the same prompt with torch's fused SDPA (library
+    flash / memory-efficient / cuDNN kernels, never the materialising math path), for
+    context next to the sparse prefill; None if no fused kernel takes the shape."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    import torch.nn.functional as F
+    n, batch, h_q, C, d = q.shape
+    qd = q.permute(1, 2, 0, 3, 4).reshape(batch, h_q, n * C, d)
+    kd = k_new.permute(1, 2, 0, 3, 4).reshape(batch, k_new.shape[2], n * C, d)
+    vd = v_new.permute(1, 2, 0, 3, 4).reshape(batch, v_new.shape[2], n * C, d)
+    try:
+        with sdpa_kernel([SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION,
+                          SDPBackend.CUDNN_ATTENTION]):
+            F.scaled_dot_product_attention(qd, kd, vd, is_causal=True, enable_gqa=True)
+            torch.cuda.synchronize()
+            ms = []
+            for _ in range(steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                F.scaled_dot_product_attention(qd, kd, vd, is_causal=True, enable_gqa=True)
+                b.record()
+                torch.cuda.synchronize()
+                ms.append(a.elapsed_time(b))
+        return statistics.median(ms)
+    except RuntimeError as e:
+        print(f"dense reference unavailable: {str(e).splitlines()[0]}", file=sys.stderr)
+        return None
+
+
+def run_prefill(args, w):
+    from query_oriented_sparse_b200 import binding as Bd
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--prefill times one prompt on one GPU")
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks, peak_src = load_peaks()
+    t = W.generate(w)
+    q, kn, vn = prompt_inputs(w, t, dev)
+    k = torch.zeros_like(t.k_cache, device=dev)
+    v = torch.zeros_like(t.v_cache, device=dev)
+    budgets = w.budgets_of_chunks()
+    b_max = max(max(budgets), 1)
+    shape = Bd.make_shape(w.batch, w.h_q, w.h_kv, w.head_dim, w.chunk, w.torch_dtype)
+    ws = torch.empty(Bd.prefill_workspace_size(shape, w.prompt_chunks, w.nq, b_max),
+                     dtype=torch.uint8, device=dev)
+    idx = torch.empty(w.batch, w.h_kv, b_max, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def prompt():
+        Bd.quoka_prefill(q, kn, vn, k, v, t.kv_off, w.nq, budgets, idx, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        prompt()
+    torch.cuda.synchronize()
+    assert Bd.device_error() == 0
+    ms = []
+    with ClockSampler(0) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            prompt()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+    assert Bd.device_error() == 0
+    ttft = statistics.median(ms)
+    tokens = w.batch * w.chunk * w.prompt_chunks
+    st = prompt_stage_model(w)
+    rl = roofline_us(st, peaks)
+    roof_ms = sum(rl.values()) / 1e3
+    dense_ms = dense_reference_ms(q, kn, vn, max(1, min(args.steps, 3)), flush)
+    n_sel = sum(1 for c, bgt in enumerate(budgets) if c > 0 and bgt > 0)
+    line = {
+        "metric": PREFILL_METRIC, "value": ttft, "unit": "ms", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ttft,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "chunk": w.chunk,
+                   "chunks": w.prompt_chunks, "prompt_tokens": w.chunk * w.prompt_chunks,
+                   "h_q": w.h_q, "h_kv": w.h_kv, "head_dim": w.head_dim, "nq": w.nq,
+                   "budget_per_chunk": "c * chunk / 8",
+                   "l2": "256 MB flush before every timed prompt"},
+        "tokens_per_s": tokens / (ttft / 1e3),
+        "gpu_launches": (2 * w.prompt_chunks + 3 * n_sel) * args.steps,
+        "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ttft,
+                          "peak_source": f"{peak_src} bf16 dense (burst) and HBM copy"},
+        "dense_sdpa_ms": dense_ms,
+        "ttft_reduction_vs_dense": (dense_ms / ttft) if dense_ms else None,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -447,7 +593,13 @@ def main():
     ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", nargs="?", const="prompt_128k", choices=sorted(W.PROMPTS),
+                    help="time a whole prompt through the prefill call (time to first token)")
     args = ap.parse_args()
+    if args.prefill:
+        if args.impl != "ours":
+            raise SystemExit("--prefill has no reference arm")
+        return run_prefill(args, W.PROMPTS[args.prefill])
     w = W.WORKLOADS[args.workload]
     if w.prompt_chunks != 1:
         raise SystemExit("bench.py times single-chunk workloads")

@@ -156,6 +156,53 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk,
 size_t sparse_chunk_attn_workspace_size(const quoka_shape* shape, int b_max);
 
 /*
+ * quoka_prefill - a whole prompt through chunked prefill, chunk after chunk, with the
+ * KV cache append inside the call (QUOKA page, Figure 1(a): the prompt is cut into
+ * chunks of C tokens; each chunk first sub-selects the cache built by the chunks before
+ * it and then runs dense attention over the compacted cache; the page's results
+ * summary reports the time to first token this loop saves on NVIDIA GPUs).
+ *
+ * Every sequence of the batch holds a prompt of n_chunks * C tokens.  For chunk
+ * c = 0 .. n_chunks-1, with P = c * C:
+ *   1. this chunk's K/V rows are written to cache rows kv_off[b] + P + t (for bf16
+ *      inside the compaction pass that the attention makes anyway, so the rows are
+ *      read from k_new / v_new once);
+ *   2. if c > 0 and budgets[c] > 0: quoka_select over the P prefix rows;
+ *   3. sparse_chunk_attn of the chunk's queries, with budget[b] = budgets[c].
+ * Chunk c's output equals quoka_select + sparse_chunk_attn called by hand with
+ * prefix_len = c * C after the caller appended chunk c's rows.
+ *
+ *   n_chunks    chunks in the prompt, >= 1
+ *   q           device, [n_chunks, batch, h_q, chunk, head_dim]
+ *   k_new       device, [n_chunks, batch, h_kv, chunk, head_dim]: the prompt's keys
+ *   v_new       device, [n_chunks, batch, h_kv, chunk, head_dim]: the prompt's values
+ *   k_cache     device, [h_kv, kv_off[batch], head_dim]; written: rows kv_off[b] ..
+ *               kv_off[b] + n_chunks*C - 1 of every KV head; other rows are untouched
+ *   v_cache     device, as k_cache
+ *   kv_off      host, batch + 1 nondecreasing row offsets, kv_off[0] >= 0,
+ *               kv_off[b+1] - kv_off[b] >= n_chunks * chunk
+ *   nq          kept queries per query head, >= 1
+ *   budgets     host, n_chunks entries, 0 <= budgets[c] <= b_max: prefix keys each
+ *               chunk keeps (chunk 0 has no prefix and ignores its entry)
+ *   b_max       row length of idx, >= 1
+ *   idx         device int32 [batch, h_kv, b_max]: scratch for the selections; holds
+ *               the last chunk's selection after the call (if it ran one)
+ *   out         device, [n_chunks, batch, h_q, chunk, head_dim]; must not alias an input
+ *   workspace   device scratch of quoka_prefill_workspace_size(shape, n_chunks, nq,
+ *               b_max) bytes; contents on entry ignored
+ * All arguments are checked before the first launch; a failed check launches nothing.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+quoka_status quoka_prefill(const quoka_shape* shape, int n_chunks, const void* q,
+                           const void* k_new, const void* v_new, void* k_cache,
+                           void* v_cache, const int64_t* kv_off, int nq,
+                           const int32_t* budgets, int b_max, int32_t* idx, void* out,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device scratch quoka_prefill() needs (0 if the arguments are invalid). */
+size_t quoka_prefill_workspace_size(const quoka_shape* shape, int n_chunks, int nq, int b_max);
+
+/*
  * quoka_select_noalloc - quoka_select without a caller-provided workspace.
  *
  * The paper has no counterpart to this call; it exists for callers that cannot

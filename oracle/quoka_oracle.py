@@ -34,6 +34,10 @@ set, so the oracle follows the method's steps in the pages' order:
    attends to the selected prefix keys of KV head h // G plus the chunk's own
    keys P .. P+t (causal), softmax(q k^T / sqrt(d)) v.
 
+7. whole-prompt chunked prefill (Figure 1(a): a prompt cut into chunks, each chunk
+   sub-selecting the cache that the chunks before it wrote): chunk c has prefix
+   P = c * C, selects over rows 0 .. P-1 with that chunk's budget, and attends.
+
 Readings where the pages are silent (each is listed with its reason in the design
 notes of the repository): the budget B counts prefix keys only and the chunk's own
 causal keys are always attended; the mean query is per query head and over
@@ -54,6 +58,7 @@ import numpy as np
 __all__ = [
     "unit_rows", "mean_query", "query_cosines", "subselect_queries", "pooled_key_scores",
     "top_budget", "select_chunk", "attend_chunk", "select_batch", "attend_batch",
+    "prefill_prompt",
 ]
 
 
@@ -245,3 +250,30 @@ def attend_batch(q, k_cache, v_cache, kv_off, prefix_len, idx_per_seq):
     return np.stack([attend_chunk(q[b], _seq_rows(k_cache, kv_off, b),
                                   _seq_rows(v_cache, kv_off, b), prefix_len[b], idx_per_seq[b])
                      for b in range(len(prefix_len))])
+
+
+def prefill_prompt(q_prompt, k_prompt, v_prompt, chunk: int, nq: int,
+                   budgets: Sequence[int]) -> Dict[str, object]:
+    """Step 7 for one sequence: the chunk loop of Figure 1(a) over a whole prompt.
+
+    q_prompt [H_q, n*C, d]; k_prompt, v_prompt [H_kv, n*C, d] (the prompt's own K/V,
+    row t written by chunk t // C); budgets has one entry per chunk.  Chunk c runs
+    steps 1-6 with P = c * C: it can only see rows the earlier chunks appended, plus
+    its own rows causally.  Returns out [H_q, n*C, d] and, per chunk, the selection.
+    """
+    q = _f64(q_prompt)
+    k = _f64(k_prompt)
+    v = _f64(v_prompt)
+    n_tok = q.shape[1]
+    C = int(chunk)
+    n = n_tok // C
+    assert n * C == n_tok and len(budgets) == n
+    out = np.zeros_like(q)
+    idx = []
+    for c in range(n):
+        P = c * C
+        qc = q[:, P:P + C]
+        sel = select_chunk(qc, k[:, :P], P, nq, int(budgets[c]))
+        out[:, P:P + C] = attend_chunk(qc, k[:, :P + C], v[:, :P + C], P, sel["idx"])
+        idx.append(sel["idx"])
+    return {"out": out, "idx": idx}

@@ -48,6 +48,11 @@ SIGNATURES = {
     "quoka_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "quoka_select_noalloc": (ctypes.c_int, [_SHAPE_P, _P, _P, _I64P, _I32P, ctypes.c_int, _I32P,
                                             ctypes.c_int, _P, _P, _P]),
+    "quoka_prefill": (ctypes.c_int, [_SHAPE_P, ctypes.c_int, _P, _P, _P, _P, _P, _I64P,
+                                     ctypes.c_int, _I32P, ctypes.c_int, _P, _P, _P,
+                                     ctypes.c_size_t, _P]),
+    "quoka_prefill_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int, ctypes.c_int,
+                                                       ctypes.c_int]),
 }
 
 _lib = None
@@ -198,6 +203,37 @@ def sparse_chunk_attn(q_chunk: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
         ctypes.byref(shape), _ptr(q_chunk), _ptr(k_cache), _ptr(v_cache), _host_i64(kv_off),
         _host_i32(prefix_len), _host_i32(budget), _ptr(idx), b_max, _ptr(out), _ptr(workspace),
         ws_bytes, ctypes.c_void_p(_stream(stream))))
+    return out
+
+
+def prefill_workspace_size(shape: QuokaShape, n_chunks: int, nq: int, b_max: int) -> int:
+    return int(lib().quoka_prefill_workspace_size(ctypes.byref(shape), int(n_chunks), int(nq),
+                                                  int(b_max)))
+
+
+def quoka_prefill(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                  k_cache: torch.Tensor, v_cache: torch.Tensor, kv_off: Sequence[int], nq: int,
+                  budgets: Sequence[int], idx: torch.Tensor, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """A whole prompt through chunked prefill, appending its K/V rows to the cache.
+
+    q [n_chunks, batch, h_q, C, d]; k_new, v_new [n_chunks, batch, h_kv, C, d];
+    budgets has one entry per chunk; returns out [n_chunks, batch, h_q, C, d].
+    """
+    n_chunks, batch, h_q, chunk, d = q.shape
+    shape = make_shape(batch, h_q, k_cache.shape[0], d, chunk, q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    b_max = int(idx.shape[-1])
+    if workspace is None:
+        n = prefill_workspace_size(shape, n_chunks, nq, b_max)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().quoka_prefill(
+        ctypes.byref(shape), int(n_chunks), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+        _ptr(v_cache), _host_i64(kv_off), int(nq), _host_i32(budgets), b_max, _ptr(idx),
+        _ptr(out), _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(stream))))
     return out
 
 

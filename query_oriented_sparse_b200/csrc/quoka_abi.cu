@@ -8,6 +8,7 @@
 #include <mutex>
 #include <string>
 #include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "qsub.cuh"
@@ -313,7 +314,8 @@ size_t attn_ws_bytes(const Dims& d, int b_max) {
 template <int D>
 quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                             const void* k, const void* v, const int32_t* idx, int b_max,
-                            void* out, unsigned char* ws, cudaStream_t st) {
+                            void* out, unsigned char* ws, cudaStream_t st,
+                            const void* k_new = nullptr, const void* v_new = nullptr) {
   AttnTcParams p;
   p.h_q = d.h_q;
   p.h_kv = d.h_kv;
@@ -333,7 +335,9 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
   const int cgrid = (int)std::min<long long>((vecs + CPT_THREADS - 1) / CPT_THREADS, (long long)sm_count() * 16);
   compact_kv_kernel<D><<<cgrid, CPT_THREADS, 0, st>>>(
       reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), rows, tab, d.h_kv, d.C,
-      b_max, p.kc_stride, idx, reinterpret_cast<uint4*>(kc), reinterpret_cast<uint4*>(vc), vecs);
+      b_max, p.kc_stride, idx, reinterpret_cast<uint4*>(kc), reinterpret_cast<uint4*>(vc), vecs,
+      reinterpret_cast<const uint4*>(k_new), reinterpret_cast<const uint4*>(v_new),
+      reinterpret_cast<uint4*>(const_cast<void*>(k)), reinterpret_cast<uint4*>(const_cast<void*>(v)));
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "compact launch");
   // 2. dense attention over it
   CUtensorMap qmap, kmap, vmap;
@@ -370,12 +374,25 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
   return QUOKA_OK;
 }
 
+// k_new / v_new (this chunk's new K/V rows, [batch, h_kv, C, d]) or NULL: when given, the
+// rows are also appended to the cache, inside the compaction pass where there is one.
 template <typename T, int D>
 quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                          const void* k, const void* v, const int32_t* idx, int b_max, void* out,
-                         unsigned char* ws, cudaStream_t st) {
-  if (d.dt == QUOKA_BF16) return launch_attn_tc<D>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
+                         unsigned char* ws, cudaStream_t st, const void* k_new = nullptr,
+                         const void* v_new = nullptr) {
+  if (d.dt == QUOKA_BF16) return launch_attn_tc<D>(d, tab, rows, q, k, v, idx, b_max, out, ws, st, k_new, v_new);
   cudaError_t e;
+  if (k_new) {
+    const int vpr = D * (int)sizeof(T) / 16;
+    const long long vecs = (long long)d.batch * d.h_kv * d.C * vpr;
+    const int agrid = (int)std::min<long long>((vecs + CPT_THREADS - 1) / CPT_THREADS, (long long)sm_count() * 16);
+    append_kv_kernel<<<agrid, CPT_THREADS, 0, st>>>(
+        reinterpret_cast<const uint4*>(k_new), reinterpret_cast<const uint4*>(v_new),
+        reinterpret_cast<uint4*>(const_cast<void*>(k)), reinterpret_cast<uint4*>(const_cast<void*>(v)),
+        rows, tab, d.h_kv, d.C, vpr, vecs);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "append launch");
+  }
   const int s = attn_simt_smem_bytes<D>();
   if ((e = ensure_smem(attn_simt_kernel<T, D>, s)) != cudaSuccess) return cuda_fail(e, "attn smem");
   dim3 grid((d.C + ATS_ROWS - 1) / ATS_ROWS, d.h_q, d.batch);
@@ -384,6 +401,38 @@ quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, con
       reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(k), reinterpret_cast<const T*>(v),
       rows, tab, d.h_q, d.h_kv, d.C, idx, b_max, reinterpret_cast<T*>(out), scale_log2);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn launch");
+  return QUOKA_OK;
+}
+
+// Whole-prompt chunked prefill: chunk c appends its K/V rows (fused with the compaction
+// where there is one), selects over the c * C rows written before it, and attends.
+template <typename T, int D>
+quoka_status run_prefill(const Dims& d, int n_chunks, const unsigned char* q, const unsigned char* k_new,
+                         const unsigned char* v_new, void* k_cache, void* v_cache, const int64_t* kv_off,
+                         int nq, const int32_t* budgets, int b_max, int32_t* idx, unsigned char* out,
+                         unsigned char* ws, unsigned char* aws, cudaStream_t st) {
+  const size_t q_chunk = (size_t)d.batch * d.h_q * d.C * d.D * d.esz;
+  const size_t kv_chunk = (size_t)d.batch * d.h_kv * d.C * d.D * d.esz;
+  std::vector<int32_t> prefix(d.batch), budget(d.batch);
+  for (int c = 0; c < n_chunks; ++c) {
+    for (int b = 0; b < d.batch; ++b) {
+      prefix[b] = c * d.C;
+      budget[b] = budgets[c];
+    }
+    SeqTable tab;
+    long long rows = 0;
+    quoka_status s = build_table(d, kv_off, prefix.data(), budget.data(), b_max, &tab, &rows);
+    if (s != QUOKA_OK) return s;
+    const unsigned char* qc = q + c * q_chunk;
+    if (c > 0 && budgets[c] > 0) {
+      const WsLayout w = ws_layout(d, tab.max_prefix, nq);
+      s = launch_select<T, D>(d, tab, rows, qc, k_cache, nq, b_max, idx, nullptr, ws, w, st);
+      if (s != QUOKA_OK) return s;
+    }
+    s = launch_attn<T, D>(d, tab, rows, qc, k_cache, v_cache, idx, b_max, out + c * q_chunk, aws, st,
+                          k_new + c * kv_chunk, v_new + c * kv_chunk);
+    if (s != QUOKA_OK) return s;
+  }
   return QUOKA_OK;
 }
 
@@ -482,6 +531,62 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk, co
   }
   return d.D == 64 ? launch_attn<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st)
                    : launch_attn<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st);
+}
+
+size_t quoka_prefill_workspace_size(const quoka_shape* shape, int n_chunks, int nq, int b_max) {
+  Dims d;
+  if (check_shape(shape, &d) != QUOKA_OK || n_chunks < 1 || nq < 1 || b_max < 1) return 0;
+  const long long max_prefix = (long long)(n_chunks - 1) * d.C;
+  if (max_prefix > (1LL << 30)) return 0;
+  return align_up(ws_layout(d, (int)max_prefix, nq).total, 256) + attn_ws_bytes(d, b_max);
+}
+
+quoka_status quoka_prefill(const quoka_shape* shape, int n_chunks, const void* q, const void* k_new,
+                           const void* v_new, void* k_cache, void* v_cache, const int64_t* kv_off,
+                           int nq, const int32_t* budgets, int b_max, int32_t* idx, void* out,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (n_chunks < 1) return fail(QUOKA_ERR_INVALID_ARG, "n_chunks must be >= 1 (got %d)", n_chunks);
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !kv_off || !budgets || !idx || !out)
+    return fail(QUOKA_ERR_INVALID_ARG,
+                "q, k_new, v_new, k_cache, v_cache, kv_off, budgets, idx and out must be non-NULL");
+  if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16) || !aligned(idx, 16) || !aligned(out, 16))
+    return fail(QUOKA_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (out == q || out == k_new || out == v_new || out == k_cache || out == v_cache)
+    return fail(QUOKA_ERR_INVALID_ARG, "out must not alias an input");
+  if (nq < 1) return fail(QUOKA_ERR_INVALID_ARG, "nq must be >= 1 (got %d)", nq);
+  if (b_max < 1) return fail(QUOKA_ERR_INVALID_ARG, "b_max must be >= 1 (got %d)", b_max);
+  const long long rows_needed = (long long)n_chunks * d.C;
+  if (rows_needed > (1LL << 30))
+    return fail(QUOKA_ERR_UNSUPPORTED, "a prompt of %lld tokens is too long", rows_needed);
+  for (int c = 0; c < n_chunks; ++c)
+    if (budgets[c] < 0 || budgets[c] > b_max)
+      return fail(QUOKA_ERR_INVALID_ARG, "budgets[%d] = %d outside [0, b_max=%d]", c, budgets[c], b_max);
+  if (kv_off[0] < 0) return fail(QUOKA_ERR_INVALID_ARG, "kv_off[0] must be >= 0");
+  for (int b = 0; b < d.batch; ++b)
+    if (kv_off[b + 1] - kv_off[b] < rows_needed)
+      return fail(QUOKA_ERR_INVALID_ARG, "sequence %d owns %lld cache rows, fewer than the prompt's %lld",
+                  b, (long long)(kv_off[b + 1] - kv_off[b]), rows_needed);
+  const size_t sel_bytes = align_up(ws_layout(d, (int)((n_chunks - 1) * d.C), nq).total, 256);
+  const size_t need = sel_bytes + attn_ws_bytes(d, b_max);
+  if (!workspace) return fail(QUOKA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (!aligned(workspace, 256)) return fail(QUOKA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < need) return fail(QUOKA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* ws = reinterpret_cast<unsigned char*>(workspace);
+  auto* aws = ws + sel_bytes;
+  const auto* qb = reinterpret_cast<const unsigned char*>(q);
+  const auto* kn = reinterpret_cast<const unsigned char*>(k_new);
+  const auto* vn = reinterpret_cast<const unsigned char*>(v_new);
+  auto* ob = reinterpret_cast<unsigned char*>(out);
+  if (d.dt == QUOKA_F32)
+    return d.D == 64 ? run_prefill<float, 64>(d, n_chunks, qb, kn, vn, k_cache, v_cache, kv_off, nq, budgets, b_max, idx, ob, ws, aws, st)
+                     : run_prefill<float, 128>(d, n_chunks, qb, kn, vn, k_cache, v_cache, kv_off, nq, budgets, b_max, idx, ob, ws, aws, st);
+  return d.D == 64 ? run_prefill<__nv_bfloat16, 64>(d, n_chunks, qb, kn, vn, k_cache, v_cache, kv_off, nq, budgets, b_max, idx, ob, ws, aws, st)
+                   : run_prefill<__nv_bfloat16, 128>(d, n_chunks, qb, kn, vn, k_cache, v_cache, kv_off, nq, budgets, b_max, idx, ob, ws, aws, st);
 }
 
 }  // extern "C"

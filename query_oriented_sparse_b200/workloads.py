@@ -16,14 +16,19 @@ results section):
     ragged_8      8 sequences, prefix ~ U[4096, 65536], chunk 1024, H_q=64, H_kv=4,
                   d=128, Nq=64, B = 12 % of each prefix rounded to 64, bf16
 
+and one whole prompt for the prefill call (chunk after chunk, cache appended inside):
+
+    prompt_128k   the ctx_128k shapes from the first token: 33 chunks of 4096, chunk c
+                  keeping c * 4096 / 8 prefix keys (its last chunk is the ctx_128k step)
+
 Value recipes (all drawn in fp32 from ``torch.Generator('cpu').manual_seed(seed)``
 and then rounded once to the workload dtype):
 
     gauss   Q, K, V ~ N(0, 1)
     rank4   Q, K ~ N(0, 1) + 2 * U_g z, with U_g an orthonormal d x 4 basis per KV
             head (QR of a Gaussian) and z ~ N(0, I_4) per token and head; V ~ N(0, 1)
-    heavy   N(0, 1), then per (sequence, KV head) 2 % of the prefix rows (without
-            replacement) are replaced by 3 * sqrt(d) * q_hat, q_hat the direction of a
+    heavy   N(0, 1), then per (sequence, KV head) 2 % of the prefix rows (of a whole
+            prompt: of all its rows) (without replacement) are replaced by 3 * sqrt(d) * q_hat, q_hat the direction of a
             uniformly drawn chunk query of a uniformly drawn head of that group
 
 KV cache layout: ``k_cache``/``v_cache`` are [H_kv, kv_total, d]; sequence b owns rows
@@ -53,6 +58,7 @@ class Workload:
     seed: int
     recipe: str                      # "gauss", "rank4" or "heavy"
     prompt_chunks: int = 1           # >1: whole prompt of prompt_chunks * chunk tokens
+    chunk_budget: Tuple[int, ...] = ()   # whole prompts: budget of each chunk (else `budget`)
 
     @property
     def batch(self) -> int:
@@ -73,6 +79,12 @@ class Workload:
     def seq_rows(self) -> Tuple[int, ...]:
         """Rows each sequence owns in the cache (prefix plus every chunk it will run)."""
         return tuple(p + self.chunk * self.prompt_chunks for p in self.prefix)
+
+    def budgets_of_chunks(self) -> Tuple[int, ...]:
+        """Budget of each chunk of a whole prompt (every sequence uses the same)."""
+        if self.chunk_budget:
+            return self.chunk_budget
+        return (self.budget[0],) * self.prompt_chunks
 
     def chunk_steps(self):
         """(chunk index, per-sequence prefix lengths) for every chunk step of the workload."""
@@ -107,16 +119,26 @@ WORKLOADS: Dict[str, Workload] = {
 # The headline single-GPU workload (128K context).
 HEADLINE = "ctx_128k"
 
+# Whole prompts run chunk by chunk through the prefill call (kept apart from WORKLOADS,
+# whose entries are single chunk steps).  prompt_128k is the 128K-context workload's
+# prompt from its first token: 33 chunks of 4096, chunk c keeping 1/8 of its c * 4096
+# prefix keys, so its last chunk is the ctx_128k step (prefix 131072, B 16384).
+PROMPTS: Dict[str, Workload] = {
+    "prompt_128k": Workload("prompt_128k", 32, 8, 128, 4096, (0,), 128, (16384,), "bf16", 3,
+                            "heavy", prompt_chunks=33,
+                            chunk_budget=tuple(c * 4096 // 8 for c in range(33))),
+}
+
 
 def custom(name: str = "custom", *, h_q: int, h_kv: int, head_dim: int, chunk: int,
            prefix, nq: int, budget, dtype: str = "bf16", seed: int = 0,
-           recipe: str = "gauss", prompt_chunks: int = 1) -> Workload:
+           recipe: str = "gauss", prompt_chunks: int = 1, chunk_budget=()) -> Workload:
     """A small ad-hoc workload (tests use these for edge cases)."""
     prefix = tuple(int(p) for p in (prefix if hasattr(prefix, "__len__") else (prefix,)))
     if not hasattr(budget, "__len__"):
         budget = (int(budget),) * len(prefix)
     return Workload(name, h_q, h_kv, head_dim, chunk, prefix, nq, tuple(int(b) for b in budget),
-                    dtype, seed, recipe, prompt_chunks)
+                    dtype, seed, recipe, prompt_chunks, tuple(int(x) for x in chunk_budget))
 
 
 @dataclasses.dataclass
@@ -163,7 +185,7 @@ def generate(w: Workload) -> Tensors:
     elif w.recipe == "heavy":
         scale = 3.0 * math.sqrt(d)
         for b in range(w.batch):
-            p = w.prefix[b]
+            p = w.prefix[b] if w.prompt_chunks == 1 else rows[b]   # candidate rows
             n_heavy = int(round(0.02 * p))
             if n_heavy == 0:
                 continue

@@ -260,10 +260,85 @@ def pin_gqa_is_independent_mqa(seed=7):
         np.testing.assert_allclose(og, o[g * G:(g + 1) * G], atol=0)
 
 
+def _sdpa_masked(q, k, v, mask_of_head):
+    """Library attention (fp64 torch SDPA) per query head with an explicit bool mask."""
+    H_q, H_kv = q.shape[0], k.shape[0]
+    G = H_q // H_kv
+    out = np.zeros(q.shape)
+    for h in range(H_q):
+        g = h // G
+        out[h] = F.scaled_dot_product_attention(
+            torch.as_tensor(q[h])[None, None], torch.as_tensor(k[g])[None, None],
+            torch.as_tensor(v[g])[None, None], attn_mask=mask_of_head(g))[0, 0].numpy()
+    return out
+
+
+def _prompt(seed, H_q=4, H_kv=2, C=5, n=4, d=8):
+    rng = np.random.default_rng(seed)
+    T = C * n
+    return (rng.normal(size=(H_q, T, d)), rng.normal(size=(H_kv, T, d)),
+            rng.normal(size=(H_kv, T, d)), C, n)
+
+
+def pin_prefill_full_budget_is_causal(seed=11):
+    """Figure 1(a) with a budget covering every prefix key: the chunk loop over the
+    whole prompt equals plain causal attention over the prompt."""
+    q, k, v, C, n = _prompt(seed)
+    T = C * n
+    res = O.prefill_prompt(q, k, v, C, 2, [T] * n)
+    causal = torch.ones(T, T, dtype=torch.bool).tril()
+    np.testing.assert_allclose(res["out"], _sdpa_masked(q, k, v, lambda g: causal),
+                               rtol=1e-12, atol=1e-13)
+
+
+def pin_prefill_zero_budget_is_block_causal(seed=12):
+    """Budget 0: every chunk attends only to itself, causally (block-diagonal mask)."""
+    q, k, v, C, n = _prompt(seed)
+    T = C * n
+    res = O.prefill_prompt(q, k, v, C, 2, [0] * n)
+    blk = torch.arange(T) // C
+    mask = (blk[:, None] == blk[None, :]) & torch.ones(T, T, dtype=torch.bool).tril()
+    np.testing.assert_allclose(res["out"], _sdpa_masked(q, k, v, lambda g: mask),
+                               rtol=1e-12, atol=1e-13)
+
+
+def pin_prefill_is_causal_over_chunks(seed=13):
+    """A partial budget: chunk c keeps min(B_c, c*C) keys of rows written before it,
+    its output is attention over exactly those keys plus its own causal keys, and
+    nothing in later chunks (their queries, keys or values) changes it."""
+    q, k, v, C, n = _prompt(seed)
+    T = C * n
+    budgets = [3, 2, 4, 7]
+    res = O.prefill_prompt(q, k, v, C, 2, budgets)
+    for c in range(n):
+        P = c * C
+        for sel in res["idx"][c]:
+            assert sel.size == min(budgets[c], P)
+            assert ((sel >= 0) & (sel < P)).all()
+        def mask_of(g, c=c, P=P):
+            m = torch.zeros(T, T, dtype=torch.bool)
+            m[:, torch.as_tensor(res["idx"][c][g], dtype=torch.long)] = True
+            m[:, P:P + C] = torch.ones(T, C, dtype=torch.bool).tril(diagonal=-P)[:, :]
+            return m[P:P + C]
+        ref = _sdpa_masked(q[:, P:P + C], k, v, mask_of)
+        np.testing.assert_allclose(res["out"][:, P:P + C], ref, rtol=1e-12, atol=1e-13)
+    rng = np.random.default_rng(seed + 100)
+    cut = 2 * C                              # chunks 2 and 3 get new content
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for x in (q2, k2, v2):
+        x[:, cut:] = rng.normal(size=x[:, cut:].shape)
+    res2 = O.prefill_prompt(q2, k2, v2, C, 2, budgets)
+    np.testing.assert_array_equal(res2["out"][:, :cut], res["out"][:, :cut])
+    for c in range(2):
+        for a, b in zip(res2["idx"][c], res["idx"][c]):
+            assert a.tolist() == b.tolist()
+
+
 ALL_PINS = [pin_query_cosine_closed_form, pin_subselect_brute_force, pin_query_scale_invariance,
             pin_scoring_closed_forms, pin_key_scale_and_permutation, pin_top_budget_brute_force,
             pin_worked_example, pin_attention_vs_sdpa, pin_full_budget_is_full_causal,
-            pin_gqa_is_independent_mqa]
+            pin_gqa_is_independent_mqa, pin_prefill_full_budget_is_causal,
+            pin_prefill_zero_budget_is_block_causal, pin_prefill_is_causal_over_chunks]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
@@ -421,9 +496,32 @@ def _mut_causal_excludes_self(mp):
     mp.setattr(O, "attend_chunk", bad)
 
 
+def _mut_prefill_own_chunk_candidates(mp):
+    """Chunk c's own rows also offered to the selection as prefix candidates."""
+    def bad(q, k, v, chunk, nq, budgets):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        out = np.zeros_like(q)
+        idx = []
+        for c in range(q.shape[1] // chunk):
+            P = c * chunk
+            sel = O.select_chunk(q[:, P:P + chunk], k[:, :P + chunk], P + chunk, nq, budgets[c])
+            out[:, P:P + chunk] = O.attend_chunk(q[:, P:P + chunk], k, v, P, sel["idx"])
+            idx.append(sel["idx"])
+        return {"out": out, "idx": idx}
+    mp.setattr(O, "prefill_prompt", bad)
+
+
+def _mut_prefill_budget_shift(mp):
+    """Each chunk run with the previous chunk's budget."""
+    orig = O.prefill_prompt
+    mp.setattr(O, "prefill_prompt", lambda q, k, v, chunk, nq, budgets:
+               orig(q, k, v, chunk, nq, [budgets[0]] + list(budgets[:-1])))
+
+
 MUTANTS = [_mut_most_similar, _mut_raw_mean, _mut_max_over_group, _mut_mean_then_max,
            _mut_no_key_norm, _mut_ties_high_index, _mut_no_softmax_scale,
-           _mut_causal_excludes_self]
+           _mut_causal_excludes_self, _mut_prefill_own_chunk_candidates,
+           _mut_prefill_budget_shift]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)
