@@ -127,7 +127,11 @@ quoka_status quoka_select(const quoka_shape* shape, const void* q_chunk, const v
  * that selected it - here the G query heads of a KV head share one selection).
  * For bf16 the call first writes that compacted cache (per sequence and KV head: the
  * selected rows, then the chunk's own rows) into `workspace`, then runs the dense
- * kernel over it; fp32 gathers rows directly and needs no workspace.
+ * kernel over it; fp32 gathers rows directly and needs no workspace.  When at most 16
+ * query rows share a KV head (G * chunk <= 16: a decode step, C = 1, or a short chunk;
+ * QUOKA page, results summary: the method also serves the generation phase) both dtypes
+ * instead gather the selected rows straight from the cache in a split-K kernel, whose
+ * per-split partial results go in `workspace`, and merge the splits per KV head.
  *
  * Query t of head h (KV head g = h / G) of sequence b attends to
  *     keys  { idx[b, g, i] : i < n_b }  U  { P + u : 0 <= u <= t }
@@ -152,7 +156,8 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk,
                                const int32_t* budget, const int32_t* idx, int b_max,
                                void* out, void* workspace, size_t ws_bytes, void* stream);
 
-/* Bytes of device scratch sparse_chunk_attn() needs (0 for fp32; 0 if invalid). */
+/* Bytes of device scratch sparse_chunk_attn() needs (0 if invalid; 0 for fp32 unless
+ * G * chunk <= 16). */
 size_t sparse_chunk_attn_workspace_size(const quoka_shape* shape, int b_max);
 
 /*

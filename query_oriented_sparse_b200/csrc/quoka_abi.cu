@@ -19,6 +19,7 @@
 #include "attn_tc.cuh"
 #include "attn_tc2.cuh"
 #include "compact.cuh"
+#include "attn_decode.cuh"
 
 using namespace quoka;
 
@@ -305,7 +306,24 @@ long long kc_block_rows(const Dims& d, int b_max) {
   return (long long)align_up((size_t)b_max + d.C, 128);
 }
 
+// Few query rows per KV head (decode, short chunks): the split-K gather kernel.
+bool use_decode(const Dims& d) { return d.G * d.C <= ADC_MAX_ROWS; }
+
+int decode_rows(const Dims& d) {
+  int r = 1;
+  while (r < d.G * d.C) r *= 2;
+  return r;
+}
+
+// Splits a (sequence, KV head) can have: the fewest keys per split is ADC_MIN_SPLIT.
+int decode_nsplit_ws(const Dims& d, int b_max) {
+  return (b_max + d.C + ADC_MIN_SPLIT - 1) / ADC_MIN_SPLIT;
+}
+
 size_t attn_ws_bytes(const Dims& d, int b_max) {
+  if (use_decode(d))
+    return align_up((size_t)d.batch * d.h_kv * decode_nsplit_ws(d, b_max) * decode_rows(d) *
+                        (d.D + 4) * 4, 256);
   if (d.dt != QUOKA_BF16) return 0;
   const size_t rows = (size_t)d.batch * d.h_kv * (size_t)kc_block_rows(d, b_max);
   return 2 * align_up(rows * d.D * 2, 256);
@@ -374,6 +392,52 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
   return QUOKA_OK;
 }
 
+template <typename T, int D, int R>
+quoka_status launch_attn_decode_r(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                                  const void* k, const void* v, const int32_t* idx, int b_max,
+                                  void* out, unsigned char* ws, cudaStream_t st) {
+  using Cfg = AdcCfg<T, D>;
+  long long total = 0;
+  int nmax = 0;
+  for (int b = 0; b < d.batch; ++b) {
+    total += (long long)d.h_kv * (tab.nsel[b] + d.C);
+    nmax = std::max(nmax, tab.nsel[b] + d.C);
+  }
+  // about eight CTAs per SM over the whole call, each at least ADC_MIN_SPLIT keys
+  const long long target = (long long)sm_count() * 8;
+  long long split = (total + target - 1) / target;
+  split = (split + 32 * Cfg::NW - 1) / (32 * Cfg::NW) * (32 * Cfg::NW);
+  split = std::min<long long>(std::max<long long>(split, ADC_MIN_SPLIT), ADC_MAX_SPLIT);
+  const int nsplit = (int)((nmax + split - 1) / split);
+  const int nsplit_ws = decode_nsplit_ws(d, b_max);
+  const int smem = adc_smem_bytes<T, D, R>();
+  cudaError_t e;
+  if ((e = ensure_smem(attn_decode_kernel<T, D, R>, smem)) != cudaSuccess) return cuda_fail(e, "decode smem");
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  float* part = reinterpret_cast<float*>(ws);
+  attn_decode_kernel<T, D, R><<<dim3(nsplit, d.h_kv, d.batch), Cfg::THREADS, smem, st>>>(
+      reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(k), reinterpret_cast<const T*>(v),
+      rows, tab, d.h_q, d.h_kv, d.C, idx, b_max, (int)split, nsplit_ws, scale_log2, part);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode launch");
+  attn_decode_combine_kernel<T, D, R><<<dim3(d.h_kv, d.batch), 128, 0, st>>>(
+      part, tab, d.h_q, d.h_kv, d.C, (int)split, nsplit_ws, reinterpret_cast<T*>(out));
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  return QUOKA_OK;
+}
+
+template <typename T, int D>
+quoka_status launch_attn_decode(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                                const void* k, const void* v, const int32_t* idx, int b_max,
+                                void* out, unsigned char* ws, cudaStream_t st) {
+  switch (decode_rows(d)) {
+    case 1: return launch_attn_decode_r<T, D, 1>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
+    case 2: return launch_attn_decode_r<T, D, 2>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
+    case 4: return launch_attn_decode_r<T, D, 4>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
+    case 8: return launch_attn_decode_r<T, D, 8>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
+    default: return launch_attn_decode_r<T, D, 16>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
+  }
+}
+
 // k_new / v_new (this chunk's new K/V rows, [batch, h_kv, C, d]) or NULL: when given, the
 // rows are also appended to the cache, inside the compaction pass where there is one.
 template <typename T, int D>
@@ -381,7 +445,9 @@ quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, con
                          const void* k, const void* v, const int32_t* idx, int b_max, void* out,
                          unsigned char* ws, cudaStream_t st, const void* k_new = nullptr,
                          const void* v_new = nullptr) {
-  if (d.dt == QUOKA_BF16) return launch_attn_tc<D>(d, tab, rows, q, k, v, idx, b_max, out, ws, st, k_new, v_new);
+  const bool decode = use_decode(d);
+  if (d.dt == QUOKA_BF16 && !decode)
+    return launch_attn_tc<D>(d, tab, rows, q, k, v, idx, b_max, out, ws, st, k_new, v_new);
   cudaError_t e;
   if (k_new) {
     const int vpr = D * (int)sizeof(T) / 16;
@@ -393,6 +459,7 @@ quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, con
         rows, tab, d.h_kv, d.C, vpr, vecs);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "append launch");
   }
+  if (decode) return launch_attn_decode<T, D>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
   const int s = attn_simt_smem_bytes<D>();
   if ((e = ensure_smem(attn_simt_kernel<T, D>, s)) != cudaSuccess) return cuda_fail(e, "attn smem");
   dim3 grid((d.C + ATS_ROWS - 1) / ATS_ROWS, d.h_q, d.batch);

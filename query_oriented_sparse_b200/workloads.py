@@ -4,7 +4,7 @@ This module only *draws* tensors: it holds none of the selection or attention
 arithmetic, so both the CUDA path (through the binding) and the fp64 oracle can be
 fed from it without sharing any method code.
 
-Five workloads are defined, matching the shapes of the QUOKA page's chunked-prefill
+Six workloads are defined, matching the shapes of the QUOKA page's chunked-prefill
 setting (page "Qualcomm QuoKA ...", Figure 1(a): a prompt split into chunks, each
 chunk attending over a compacted KV cache) and its ~12 % KV budget (same page,
 results section):
@@ -15,6 +15,9 @@ results section):
     ctx_128k      H_q=32, H_kv=8, d=128, prefix 131072 + chunk 4096, Nq=128, B=16384, bf16
     ragged_8      8 sequences, prefix ~ U[4096, 65536], chunk 1024, H_q=64, H_kv=4,
                   d=128, Nq=64, B = 12 % of each prefix rounded to 64, bf16
+    decode_32     one decode step of 32 sequences: prefix ~ U[2048, 16384], chunk 1 (the
+                  new token), H_q=32, H_kv=8, d=128, Nq=1, B = 12 % of each prefix
+                  rounded to 64, bf16, selection every step
 
 and one whole prompt for the prefill call (chunk after chunk, cache appended inside):
 
@@ -104,6 +107,14 @@ def _ragged_prefixes(seed: int) -> Tuple[int, ...]:
 
 _RAGGED = _ragged_prefixes(4)
 
+
+def _decode_prefixes(seed: int) -> Tuple[int, ...]:
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return tuple(int(x) for x in torch.randint(2048, 16385, (32,), generator=g))
+
+
+_DECODE = _decode_prefixes(5)
+
 WORKLOADS: Dict[str, Workload] = {
     "tiny_mqa": Workload("tiny_mqa", 4, 1, 64, 128, (0,), 16, (128,), "f32", 0, "gauss",
                          prompt_chunks=4),
@@ -114,6 +125,8 @@ WORKLOADS: Dict[str, Workload] = {
                          "heavy"),
     "ragged_8": Workload("ragged_8", 64, 4, 128, 1024, _RAGGED, 64,
                          tuple(_budget_12pct(p) for p in _RAGGED), "bf16", 4, "rank4"),
+    "decode_32": Workload("decode_32", 32, 8, 128, 1, _DECODE, 1,
+                          tuple(_budget_12pct(p) for p in _DECODE), "bf16", 5, "heavy"),
 }
 
 # The headline single-GPU workload (128K context).

@@ -1,8 +1,9 @@
-"""GPU parity on the five full-size workloads, through the same calls bench.py times.
+"""GPU parity on the six full-size workloads, through the same calls bench.py times.
 
 Selection is checked completely (every kept set, pooled score and index set, with
 near-ties counted); attention is checked on every row for the two small workloads
-and on sampled rows (plus the first and last positions) for the large ones.
+and the decode step, and on sampled rows (plus the first and last positions) for the
+large ones.
 """
 import pytest
 
@@ -17,7 +18,7 @@ pytestmark = pytest.mark.gpu
 def test_workload_parity(name, cuda_device):
     w = W.WORKLOADS[name]
     t = W.generate(w)
-    full_rows = name in ("tiny_mqa", "gqa_8k")
+    full_rows = name in ("tiny_mqa", "gqa_8k", "decode_32")
     for c, _ in w.chunk_steps():
         res = run_gpu(w, t, chunk_index=c)
         rep = check_step(w, t, res, chunk_index=c, attn_rows=None if full_rows else 96)
