@@ -41,7 +41,15 @@ from query_oriented_sparse_b200 import workloads as W  # noqa: E402
 METRIC = "chunked-prefill sparse-attn tokens/s (select+attend) and % of roofline, 1 B200"
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 5  # qsub, score, top-k, compaction, attention
+def launches_per_step(w):
+    """Kernels one step launches.  Selection: query subselect, scoring and top-k, or only
+    scoring and top-k when every query is kept and G * C <= 16 (the decode shape).
+    Attention: the gather kernel and its combine when G * C <= 16, else compaction and
+    the tensor-core kernel (bf16) or the CUDA-core kernel alone (fp32)."""
+    small = w.group * w.chunk <= 16
+    sel = 2 if small and w.nq >= w.chunk else 3
+    att = 2 if small or w.dtype == "bf16" else 1
+    return sel + att
 # DRAM traffic of one attention-kernel launch on the 128K-context workload
 # (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture, summarised in
 # profiles/attn_tc2_kernel_ctx_128k.md), valid only for the kernel sources it was taken
@@ -458,7 +466,7 @@ def run_ours(args, w):
                    "parallelism": f"independent chunk step per GPU x{world}"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": launches_per_step(w) * args.steps,
         "stage_us": {"select": statistics.mean(sel_ms) * 1e3,
                      "attn": statistics.mean(att_ms) * 1e3},
         "roofline": roof,

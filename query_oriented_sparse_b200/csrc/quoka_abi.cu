@@ -20,6 +20,7 @@
 #include "attn_tc2.cuh"
 #include "compact.cuh"
 #include "attn_decode.cuh"
+#include "select_decode.cuh"
 
 using namespace quoka;
 
@@ -112,13 +113,15 @@ struct WsLayout {
   int nk, nkp;              // kept queries per head, and that count padded to 16
   int ncg, heads_per_cg;    // column groups per KV head for the tensor-core scoring
   bool tc;                  // tensor-core scoring (bf16) or CUDA-core scoring (fp32)
+  bool dec;                 // every query kept and <= 16 rows per KV head: decode scoring
 };
 
 WsLayout ws_layout(const Dims& d, int max_prefix, int nq) {
   WsLayout w;
   w.nk = nq < d.C ? nq : d.C;
   w.nkp = (w.nk + 15) / 16 * 16;
-  w.tc = d.dt == QUOKA_BF16 && w.nkp <= STC_SLICE;
+  w.dec = w.nk == d.C && d.G * d.C <= ADC_MAX_ROWS;
+  w.tc = !w.dec && d.dt == QUOKA_BF16 && w.nkp <= STC_SLICE;
   if (w.tc) {
     // a column group is at most two head-aligned slices of <= 256 columns
     const int hmax = 2 * (STC_SLICE / w.nkp);
@@ -260,6 +263,70 @@ quoka_status launch_score_tc(const Dims& d, const SeqTable& tab, long long rows,
   return QUOKA_OK;
 }
 
+// Top-B per (sequence, KV head): one CTA per row when there are many rows short enough to
+// stage in shared memory, else a 16-CTA cluster per row.
+quoka_status launch_topk(const Dims& d, const SeqTable& tab, int b_max, int32_t* idx_out,
+                         const WsLayout& w, float* pooled, cudaStream_t st) {
+  cudaError_t e;
+  const int nrows = d.batch * d.h_kv;
+  if (tab.max_prefix <= TOPK_BLOCK_MAX_KEYS && nrows >= TOPK_BLOCK_MIN_ROWS) {
+    const int smem = std::max(tab.max_prefix, 1) * 4;
+    if ((e = ensure_smem(topk_block_kernel, smem)) != cudaSuccess) return cuda_fail(e, "topk_block smem");
+    topk_block_kernel<<<nrows, 512, smem, st>>>(pooled, w.pooled_stride, w.ncg, w.cg_stride,
+                                                 1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk_block launch");
+    return QUOKA_OK;
+  }
+  const int tk_keys = std::min((tab.max_prefix + TOPK_CS - 1) / TOPK_CS, TOPK_STAGE_KEYS);
+  const int tk_smem = tk_keys * 4;
+  if ((e = ensure_smem(topk_kernel, tk_smem)) != cudaSuccess) return cuda_fail(e, "topk smem");
+  if ((e = ensure_cluster16(topk_kernel)) != cudaSuccess) return cuda_fail(e, "topk cluster size");
+  topk_kernel<<<nrows * TOPK_CS, TOPK_THREADS, tk_smem, st>>>(
+      pooled, w.pooled_stride, w.ncg, w.cg_stride, 1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
+  return QUOKA_OK;
+}
+
+template <typename T, int D, int R>
+quoka_status launch_score_decode_r(const Dims& d, const SeqTable& tab, long long rows,
+                                   const void* q, const void* k, float* pooled, const WsLayout& w,
+                                   cudaStream_t st) {
+  const int smem = scd_smem_bytes<T, D, R>();
+  cudaError_t e;
+  if ((e = ensure_smem(score_decode_kernel<T, D, R>, smem)) != cudaSuccess) return cuda_fail(e, "score_decode smem");
+  dim3 grid((tab.max_prefix + SCD_KEYS - 1) / SCD_KEYS, d.h_kv, d.batch);
+  score_decode_kernel<T, D, R><<<grid, SCD_THREADS, smem, st>>>(
+      reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(k), rows, tab, d.h_q, d.h_kv, d.C,
+      pooled, w.pooled_stride);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score_decode launch");
+  return QUOKA_OK;
+}
+
+// Every query kept and at most 16 query rows per KV head: the kept positions are all of
+// them, and the scoring streams the prefix keys on CUDA cores.
+template <typename T, int D>
+quoka_status launch_select_decode(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                                  const void* k, int nq, int32_t* kept_out, float* pooled,
+                                  const WsLayout& w, cudaStream_t st) {
+  cudaError_t e;
+  if (kept_out) {
+    const long long n = (long long)d.batch * d.h_q * nq;
+    const int grid = (int)std::min<long long>((n + 255) / 256, (long long)sm_count() * 4);
+    kept_all_kernel<<<grid, 256, 0, st>>>(kept_out, d.batch * d.h_q, d.C, nq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "kept launch");
+  }
+  if (tab.max_prefix == 0) return QUOKA_OK;
+  int r = 1;
+  while (r < d.G * d.C) r *= 2;
+  switch (r) {
+    case 1: return launch_score_decode_r<T, D, 1>(d, tab, rows, q, k, pooled, w, st);
+    case 2: return launch_score_decode_r<T, D, 2>(d, tab, rows, q, k, pooled, w, st);
+    case 4: return launch_score_decode_r<T, D, 4>(d, tab, rows, q, k, pooled, w, st);
+    case 8: return launch_score_decode_r<T, D, 8>(d, tab, rows, q, k, pooled, w, st);
+    default: return launch_score_decode_r<T, D, 16>(d, tab, rows, q, k, pooled, w, st);
+  }
+}
+
 template <typename T, int D>
 quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                            const void* k, int nq, int b_max, int32_t* idx_out, int32_t* kept_out,
@@ -269,6 +336,12 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
   float* qbias = reinterpret_cast<float*>(ws + w.qbias);
   float* pooled = reinterpret_cast<float*>(ws + w.pooled);
   cudaError_t e;
+
+  if (w.dec) {
+    quoka_status s = launch_select_decode<T, D>(d, tab, rows, q, k, nq, kept_out, pooled, w, st);
+    if (s != QUOKA_OK) return s;
+    return launch_topk(d, tab, b_max, idx_out, w, pooled, st);
+  }
 
   const int qs_smem = d.C * 4;                 // the chunk-wide key array
   if ((e = ensure_smem(qsub_kernel<T, D>, qs_smem)) != cudaSuccess) return cuda_fail(e, "qsub smem");
@@ -291,14 +364,7 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
     }
   }
 
-  const int tk_keys = std::min((tab.max_prefix + TOPK_CS - 1) / TOPK_CS, TOPK_STAGE_KEYS);
-  const int tk_smem = tk_keys * 4;
-  if ((e = ensure_smem(topk_kernel, tk_smem)) != cudaSuccess) return cuda_fail(e, "topk smem");
-  if ((e = ensure_cluster16(topk_kernel)) != cudaSuccess) return cuda_fail(e, "topk cluster size");
-  topk_kernel<<<d.batch * d.h_kv * TOPK_CS, TOPK_THREADS, tk_smem, st>>>(
-      pooled, w.pooled_stride, w.ncg, w.cg_stride, 1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
-  return QUOKA_OK;
+  return launch_topk(d, tab, b_max, idx_out, w, pooled, st);
 }
 
 // Rows per (sequence, KV head) block of the compacted cache.
