@@ -387,21 +387,27 @@ def run_ours(args, w):
     total_s = sum(step_ms) / 1e3
     assert Bd.device_error() == 0
 
-    # end to end through host buffers: every step's new inputs (Q and the chunk's own K/V
-    # rows) go host->device from pinned memory and its output comes back device->host,
-    # pipelined as a server runs it: step i+1's inputs are uploaded on one copy stream and
-    # step i's output is read back on another while step i computes, with inputs and
-    # outputs double-buffered.  The timed region runs from the first upload to the last
-    # read-back, so every step's copies are inside it.
+    # end to end through host buffers and the serving call (quoka_step): every step's new
+    # inputs (Q and the chunk's own K/V rows, packed [batch, h_kv, C, d]) go host->device
+    # from pinned memory, the call appends the K/V rows to the cache, selects and attends,
+    # and the output comes back device->host.  Steps are pipelined as a server runs them:
+    # step i+1's inputs are uploaded on one copy stream and step i's output is read back
+    # on another while step i computes, with inputs and outputs double-buffered (the
+    # cache is written only by the steps themselves, in stream order).  The timed region
+    # runs from the first upload to the last read-back, so every step's copies are in it.
     C = w.chunk
     q_h = t.q.pin_memory()
     kv_rows = [(t.kv_off[b] + w.prefix[b], t.kv_off[b] + w.prefix[b] + C) for b in range(w.batch)]
-    kc_h = [t.k_cache[:, a:b_].contiguous().pin_memory() for a, b_ in kv_rows]
-    vc_h = [t.v_cache[:, a:b_].contiguous().pin_memory() for a, b_ in kv_rows]
+    kn_h = torch.stack([t.k_cache[:, a:b_] for a, b_ in kv_rows]).contiguous().pin_memory()
+    vn_h = torch.stack([t.v_cache[:, a:b_] for a, b_ in kv_rows]).contiguous().pin_memory()
     out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    h2d = q_h.numel() * q_h.element_size() + sum(2 * x.numel() * x.element_size() for x in kc_h)
+    h2d = sum(x.numel() * x.element_size() for x in (q_h, kn_h, vn_h))
     d2h = out_h[0].numel() * out_h[0].element_size()
-    qb, kb, vb, ob = [q, q.clone()], [k, k.clone()], [v, v.clone()], [out, torch.empty_like(out)]
+    qb, ob = [q, q.clone()], [torch.empty_like(out), torch.empty_like(out)]
+    knb = [torch.empty(kn_h.shape, dtype=kn_h.dtype, device=dev) for _ in range(2)]
+    vnb = [torch.empty(vn_h.shape, dtype=vn_h.dtype, device=dev) for _ in range(2)]
+    sws = torch.empty(Bd.step_workspace_size(shape, max(w.prefix), w.nq, b_max), dtype=torch.uint8,
+                      device=dev)
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of buffer b landed
     ev_cmp = [torch.cuda.Event() for _ in range(2)]     # the step on buffer b has finished
@@ -417,19 +423,15 @@ def run_ours(args, w):
                 if i == 0 and timed:
                     t0.record(s_in)
                 qb[b].copy_(q_h, non_blocking=True)
-                for (a, b_), kh, vh in zip(kv_rows, kc_h, vc_h):
-                    for hh in range(kh.shape[0]):          # one contiguous copy per KV head
-                        kb[b][hh, a:b_].copy_(kh[hh], non_blocking=True)
-                        vb[b][hh, a:b_].copy_(vh[hh], non_blocking=True)
+                knb[b].copy_(kn_h, non_blocking=True)
+                vnb[b].copy_(vn_h, non_blocking=True)
                 ev_in[b].record(s_in)
             stream.wait_event(ev_in[b])
             if i >= 2:
                 stream.wait_event(ev_out[b])
             flush.zero_()
-            Bd.quoka_select(qb[b], kb[b], t.kv_off, w.prefix, w.nq, w.budget, b_max, idx_out=idx,
-                            workspace=ws)
-            Bd.sparse_chunk_attn(qb[b], kb[b], vb[b], t.kv_off, w.prefix, w.budget, idx, out=ob[b],
-                                 workspace=aws)
+            Bd.quoka_step(qb[b], knb[b], vnb[b], k, v, t.kv_off, w.prefix, w.nq, w.budget, idx,
+                          out=ob[b], workspace=sws)
             ev_cmp[b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_cmp[b])
@@ -443,6 +445,7 @@ def run_ours(args, w):
     e2e_run(max(2, args.warmup), False)
     e2e_total_ms = e2e_run(args.steps, True)
     last = (args.steps - 1) & 1
+    # the serving call's output equals the two single calls' (timed above)
     assert torch.equal(out_h[last].to(dev), ob[last]) and torch.equal(ob[last], out)
 
     tokens = w.batch * C

@@ -164,6 +164,37 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk,
 size_t sparse_chunk_attn_workspace_size(const quoka_shape* shape, int b_max);
 
 /*
+ * quoka_step - one step of a chunked prefill or of decode, the way a serving loop runs
+ * it: the chunk's new K/V rows go into the cache inside the call, then quoka_select and
+ * sparse_chunk_attn run as described above (QUOKA page, Figure 1(a): each chunk sub-
+ * selects the cache written before it, then attends over the compacted cache).
+ *
+ * For every sequence b the chunk's K/V rows are written to cache rows
+ * kv_off[b] + prefix_len[b] + t (for bf16 inside the compaction pass that the attention
+ * makes anyway).  The selection reads only rows below prefix_len[b], so the result
+ * equals appending the rows by hand and calling quoka_select and sparse_chunk_attn.
+ * The selection is skipped when no sequence keeps a prefix key.
+ *
+ *   q_chunk, kv_off, prefix_len, nq, budget, b_max   as for quoka_select
+ *   k_new, v_new  device, [batch, h_kv, chunk, head_dim]: the chunk's keys and values
+ *   k_cache, v_cache  device, [h_kv, kv_off[batch], head_dim]; rows kv_off[b] +
+ *               prefix_len[b] .. + chunk - 1 are written, other rows untouched
+ *   idx         device int32 [batch, h_kv, b_max]: the selection (written when one runs)
+ *   out         device [batch, h_q, chunk, head_dim]; must not alias an input
+ *   workspace   device scratch of quoka_step_workspace_size(shape, max_b prefix_len[b],
+ *               nq, b_max) bytes; contents on entry ignored
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA; a failed check launches nothing.
+ */
+quoka_status quoka_step(const quoka_shape* shape, const void* q_chunk, const void* k_new,
+                        const void* v_new, void* k_cache, void* v_cache,
+                        const int64_t* kv_off, const int32_t* prefix_len, int nq,
+                        const int32_t* budget, int b_max, int32_t* idx, void* out,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device scratch quoka_step() needs (0 if the arguments are invalid). */
+size_t quoka_step_workspace_size(const quoka_shape* shape, int max_prefix, int nq, int b_max);
+
+/*
  * quoka_prefill - a whole prompt through chunked prefill, chunk after chunk, with the
  * KV cache append inside the call (QUOKA page, Figure 1(a): the prompt is cut into
  * chunks of C tokens; each chunk first sub-selects the cache built by the chunks before

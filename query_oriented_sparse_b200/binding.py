@@ -48,6 +48,10 @@ SIGNATURES = {
     "quoka_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "quoka_select_noalloc": (ctypes.c_int, [_SHAPE_P, _P, _P, _I64P, _I32P, ctypes.c_int, _I32P,
                                             ctypes.c_int, _P, _P, _P]),
+    "quoka_step": (ctypes.c_int, [_SHAPE_P, _P, _P, _P, _P, _P, _I64P, _I32P, ctypes.c_int,
+                                  _I32P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
+    "quoka_step_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_int]),
     "quoka_prefill": (ctypes.c_int, [_SHAPE_P, ctypes.c_int, _P, _P, _P, _P, _P, _I64P,
                                      ctypes.c_int, _I32P, ctypes.c_int, _P, _P, _P,
                                      ctypes.c_size_t, _P]),
@@ -203,6 +207,33 @@ def sparse_chunk_attn(q_chunk: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
         ctypes.byref(shape), _ptr(q_chunk), _ptr(k_cache), _ptr(v_cache), _host_i64(kv_off),
         _host_i32(prefix_len), _host_i32(budget), _ptr(idx), b_max, _ptr(out), _ptr(workspace),
         ws_bytes, ctypes.c_void_p(_stream(stream))))
+    return out
+
+
+def step_workspace_size(shape: QuokaShape, max_prefix: int, nq: int, b_max: int) -> int:
+    return int(lib().quoka_step_workspace_size(ctypes.byref(shape), int(max_prefix), int(nq),
+                                               int(b_max)))
+
+
+def quoka_step(q_chunk: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+               k_cache: torch.Tensor, v_cache: torch.Tensor, kv_off: Sequence[int],
+               prefix_len: Sequence[int], nq: int, budget: Sequence[int], idx: torch.Tensor,
+               out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One chunk (or decode) step with the cache append: q_chunk [batch, h_q, C, d],
+    k_new / v_new [batch, h_kv, C, d]; returns out [batch, h_q, C, d]."""
+    shape = shape_of(q_chunk, k_cache)
+    if out is None:
+        out = torch.empty_like(q_chunk)
+    b_max = int(idx.shape[-1])
+    if workspace is None:
+        n = step_workspace_size(shape, max(prefix_len), nq, b_max)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q_chunk.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().quoka_step(
+        ctypes.byref(shape), _ptr(q_chunk), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+        _ptr(v_cache), _host_i64(kv_off), _host_i32(prefix_len), int(nq), _host_i32(budget),
+        b_max, _ptr(idx), _ptr(out), _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(stream))))
     return out
 
 

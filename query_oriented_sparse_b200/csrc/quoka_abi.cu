@@ -537,6 +537,24 @@ quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, con
   return QUOKA_OK;
 }
 
+// One step with the append: select over each sequence's prefix (when any key is to be
+// kept), then attend, the chunk's new K/V rows going into the cache on the way (fused
+// with the compaction where there is one).
+template <typename T, int D>
+quoka_status run_step(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                      const void* k_new, const void* v_new, void* k_cache, void* v_cache, int nq,
+                      int b_max, int32_t* idx, void* out, unsigned char* ws, unsigned char* aws,
+                      cudaStream_t st) {
+  bool any = false;
+  for (int b = 0; b < d.batch; ++b) any = any || tab.nsel[b] > 0;
+  if (any) {
+    const WsLayout w = ws_layout(d, tab.max_prefix, nq);
+    quoka_status s = launch_select<T, D>(d, tab, rows, q, k_cache, nq, b_max, idx, nullptr, ws, w, st);
+    if (s != QUOKA_OK) return s;
+  }
+  return launch_attn<T, D>(d, tab, rows, q, k_cache, v_cache, idx, b_max, out, aws, st, k_new, v_new);
+}
+
 // Whole-prompt chunked prefill: chunk c appends its K/V rows (fused with the compaction
 // where there is one), selects over the c * C rows written before it, and attends.
 template <typename T, int D>
@@ -556,14 +574,8 @@ quoka_status run_prefill(const Dims& d, int n_chunks, const unsigned char* q, co
     long long rows = 0;
     quoka_status s = build_table(d, kv_off, prefix.data(), budget.data(), b_max, &tab, &rows);
     if (s != QUOKA_OK) return s;
-    const unsigned char* qc = q + c * q_chunk;
-    if (c > 0 && budgets[c] > 0) {
-      const WsLayout w = ws_layout(d, tab.max_prefix, nq);
-      s = launch_select<T, D>(d, tab, rows, qc, k_cache, nq, b_max, idx, nullptr, ws, w, st);
-      if (s != QUOKA_OK) return s;
-    }
-    s = launch_attn<T, D>(d, tab, rows, qc, k_cache, v_cache, idx, b_max, out + c * q_chunk, aws, st,
-                          k_new + c * kv_chunk, v_new + c * kv_chunk);
+    s = run_step<T, D>(d, tab, rows, q + c * q_chunk, k_new + c * kv_chunk, v_new + c * kv_chunk,
+                       k_cache, v_cache, nq, b_max, idx, out + c * q_chunk, ws, aws, st);
     if (s != QUOKA_OK) return s;
   }
   return QUOKA_OK;
@@ -664,6 +676,46 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk, co
   }
   return d.D == 64 ? launch_attn<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st)
                    : launch_attn<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st);
+}
+
+size_t quoka_step_workspace_size(const quoka_shape* shape, int max_prefix, int nq, int b_max) {
+  Dims d;
+  if (check_shape(shape, &d) != QUOKA_OK || max_prefix < 0 || nq < 1 || b_max < 1) return 0;
+  return align_up(ws_layout(d, max_prefix, nq).total, 256) + attn_ws_bytes(d, b_max);
+}
+
+quoka_status quoka_step(const quoka_shape* shape, const void* q_chunk, const void* k_new,
+                        const void* v_new, void* k_cache, void* v_cache, const int64_t* kv_off,
+                        const int32_t* prefix_len, int nq, const int32_t* budget, int b_max,
+                        int32_t* idx, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (!q_chunk || !k_new || !v_new || !k_cache || !v_cache || !idx || !out)
+    return fail(QUOKA_ERR_INVALID_ARG,
+                "q_chunk, k_new, v_new, k_cache, v_cache, idx and out must be non-NULL");
+  if (!aligned(q_chunk, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16) || !aligned(idx, 16) || !aligned(out, 16))
+    return fail(QUOKA_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (out == q_chunk || out == k_new || out == v_new || out == k_cache || out == v_cache)
+    return fail(QUOKA_ERR_INVALID_ARG, "out must not alias an input");
+  if (nq < 1) return fail(QUOKA_ERR_INVALID_ARG, "nq must be >= 1 (got %d)", nq);
+  SeqTable tab;
+  long long rows = 0;
+  if ((s = build_table(d, kv_off, prefix_len, budget, b_max, &tab, &rows)) != QUOKA_OK) return s;
+  const size_t sel_bytes = align_up(ws_layout(d, tab.max_prefix, nq).total, 256);
+  const size_t need = sel_bytes + attn_ws_bytes(d, b_max);
+  if (!workspace) return fail(QUOKA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (!aligned(workspace, 256)) return fail(QUOKA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < need) return fail(QUOKA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* ws = reinterpret_cast<unsigned char*>(workspace);
+  auto* aws = ws + sel_bytes;
+  if (d.dt == QUOKA_F32)
+    return d.D == 64 ? run_step<float, 64>(d, tab, rows, q_chunk, k_new, v_new, k_cache, v_cache, nq, b_max, idx, out, ws, aws, st)
+                     : run_step<float, 128>(d, tab, rows, q_chunk, k_new, v_new, k_cache, v_cache, nq, b_max, idx, out, ws, aws, st);
+  return d.D == 64 ? run_step<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_new, v_new, k_cache, v_cache, nq, b_max, idx, out, ws, aws, st)
+                   : run_step<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_new, v_new, k_cache, v_cache, nq, b_max, idx, out, ws, aws, st);
 }
 
 size_t quoka_prefill_workspace_size(const quoka_shape* shape, int n_chunks, int nq, int b_max) {
