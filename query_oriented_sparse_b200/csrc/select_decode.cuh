@@ -7,7 +7,7 @@
 // tensor-core tile would carry a few useful columns and pay a fixed hand-off latency per
 // tile.  So:
 //   kept_all_kernel      writes the kept positions (all of them) when the caller asks;
-//   score_decode_kernel  one CTA per (512-key tile, KV head, sequence), four warps; each
+//   score_decode_kernel  one CTA per (1024-key tile, KV head, sequence), four warps; each
 //                        warp streams batches of 32 consecutive key rows into its own
 //                        shared-memory stage with 16-byte cp.async (two stages, the next
 //                        batch in flight while this one is scored), and lane l scores key
@@ -24,7 +24,7 @@ namespace quoka {
 
 constexpr int SCD_WARPS = 4;
 constexpr int SCD_THREADS = SCD_WARPS * 32;
-constexpr int SCD_BATCHES = 4;                              // 32-key batches per warp
+constexpr int SCD_BATCHES = 8;                              // 32-key batches per warp
 constexpr int SCD_KEYS = SCD_WARPS * SCD_BATCHES * 32;      // keys per CTA
 constexpr int TOPK_BLOCK_MAX_KEYS = 32768;                  // staged keys (128 KB)
 constexpr int TOPK_BLOCK_MIN_ROWS = 32;                     // (sequence, KV head) rows
