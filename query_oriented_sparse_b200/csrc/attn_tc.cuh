@@ -88,7 +88,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   const int npairs = (p.C + 2 * p.TP - 1) / (2 * p.TP);
   const int pair = npairs - 1 - (int)blockIdx.x;           // longest key ranges first
   const int t0 = pair * 2 * p.TP;
-  const int P = tab.prefix[b], nsel = tab.nsel[b];
+  const int nsel = tab.nsel[b];
   const int tend = min(p.C, t0 + 2 * p.TP);                  // positions [t0, tend)
   const int nkeys = nsel + tend;                             // selected + chunk keys 0..tend-1
   const int nblk = (nkeys + 127) / 128;

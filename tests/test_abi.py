@@ -126,6 +126,78 @@ def test_attn_rejects(case, status):
     assert _attn(shape, **case) == status
 
 
+def _step(shape, q=FAKE, k_new=FAKE + 0x2000, v_new=FAKE + 0x3000, k=FAKE + 0x4000,
+          v=FAKE + 0x5000, kv_off=(0, 1024), prefix=(512,), nq=8, budget=(64,), b_max=64,
+          idx=FAKE + 0x6000, out=FAKE + 0x7000, ws=FAKE, ws_bytes=1 << 30):
+    return Bd.lib().quoka_step(ctypes.byref(shape), q, k_new, v_new, k, v, Bd._host_i64(kv_off),
+                               Bd._host_i32(prefix), nq, Bd._host_i32(budget), b_max, idx, out,
+                               ws, ws_bytes, None)
+
+
+@no_gpu
+@pytest.mark.parametrize("case,status", [
+    (dict(shape=dict(head_dim=96)), Bd.QUOKA_ERR_UNSUPPORTED),
+    (dict(k_new=None), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(v_new=FAKE + 0x3004), Bd.QUOKA_ERR_INVALID_ARG),       # misaligned
+    (dict(out=FAKE), Bd.QUOKA_ERR_INVALID_ARG),                  # aliases q
+    (dict(out=FAKE + 0x4000), Bd.QUOKA_ERR_INVALID_ARG),         # aliases the K cache
+    (dict(budget=(65,)), Bd.QUOKA_ERR_INVALID_ARG),              # budget > b_max
+    (dict(prefix=(900,)), Bd.QUOKA_ERR_INVALID_ARG),             # prefix + chunk > rows
+    (dict(nq=0), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(ws=None), Bd.QUOKA_ERR_WORKSPACE),
+    (dict(ws_bytes=1000), Bd.QUOKA_ERR_WORKSPACE),
+    (dict(ws=FAKE + 64), Bd.QUOKA_ERR_INVALID_ARG),              # workspace not 256-aligned
+])
+def test_step_rejects(case, status):
+    shp = dict(batch=1, h_q=8, h_kv=2, head_dim=128, chunk=256, dtype=Bd.QUOKA_BF16)
+    shp.update(case.pop("shape", {}))
+    assert _step(Bd.QuokaShape(**shp), **case) == status
+    assert Bd.lib().quoka_last_error().decode()
+
+
+def _prefill(shape, n_chunks=2, q=FAKE, k_new=FAKE + 0x2000, v_new=FAKE + 0x3000,
+             k=FAKE + 0x4000, v=FAKE + 0x5000, kv_off=(0, 1024), nq=8, budgets=(0, 64), b_max=64,
+             idx=FAKE + 0x6000, out=FAKE + 0x7000, ws=FAKE, ws_bytes=1 << 30):
+    return Bd.lib().quoka_prefill(ctypes.byref(shape), n_chunks, q, k_new, v_new, k, v,
+                                  Bd._host_i64(kv_off), nq,
+                                  None if budgets is None else Bd._host_i32(budgets), b_max, idx,
+                                  out, ws, ws_bytes, None)
+
+
+@no_gpu
+@pytest.mark.parametrize("case,status", [
+    (dict(n_chunks=0, budgets=(0,)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(budgets=(0, 65)), Bd.QUOKA_ERR_INVALID_ARG),           # budget > b_max
+    (dict(budgets=(0, -1)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(budgets=None), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(kv_off=(0, 500)), Bd.QUOKA_ERR_INVALID_ARG),           # fewer rows than the prompt
+    (dict(n_chunks=5, budgets=(0, 8, 8, 8, 8)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(out=FAKE), Bd.QUOKA_ERR_INVALID_ARG),                  # aliases q
+    (dict(q=FAKE + 2), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(ws=None), Bd.QUOKA_ERR_WORKSPACE),
+    (dict(ws_bytes=100), Bd.QUOKA_ERR_WORKSPACE),
+])
+def test_prefill_rejects(case, status):
+    shape = Bd.QuokaShape(batch=1, h_q=8, h_kv=2, head_dim=128, chunk=256, dtype=Bd.QUOKA_BF16)
+    assert _prefill(shape, **case) == status
+    assert Bd.lib().quoka_last_error().decode()
+
+
+def test_step_and_prefill_workspace_sizes():
+    s = Bd.make_shape(1, 32, 8, 128, 4096, torch.bfloat16)
+    n_step = Bd.step_workspace_size(s, 131072, 128, 16384)
+    assert n_step == (Bd.select_workspace_size(s, 131072, 128) + 255) // 256 * 256 + \
+        Bd.attn_workspace_size(s, 16384)
+    # 33 chunks: the last selects over 32 * 4096 prefix rows
+    assert Bd.prefill_workspace_size(s, 33, 128, 16384) == n_step
+    assert Bd.prefill_workspace_size(s, 0, 128, 16384) == 0
+    assert Bd.step_workspace_size(s, -1, 128, 16384) == 0
+    # decode (G * C <= 16): the attention scratch holds split partials, not a compacted cache
+    d = Bd.make_shape(32, 32, 8, 128, 1, torch.bfloat16)
+    parts = 32 * 8 * ((2048 + 1 + 255) // 256) * 4 * (128 + 4) * 4
+    assert Bd.attn_workspace_size(d, 2048) == (parts + 255) // 256 * 256
+
+
 def test_null_shape_rejected():
     lib = Bd.lib()
     assert lib.quoka_select(None, FAKE, FAKE, Bd._host_i64((0, 8)), Bd._host_i32((0,)), 1,

@@ -260,6 +260,31 @@ def pin_gqa_is_independent_mqa(seed=7):
         np.testing.assert_allclose(og, o[g * G:(g + 1) * G], atol=0)
 
 
+def pin_decode_is_mean_cosine(seed=14):
+    """A decode step (C = 1): the subselect keeps the one query, so a key's score is the
+    mean over the group's heads of its cosine with each head's query (torch's
+    cosine_similarity), the top-B follows that, and a key scaled by any positive factor
+    keeps its score."""
+    rng = np.random.default_rng(seed)
+    H_q, H_kv, P, d, B = 8, 2, 40, 16, 7
+    G = H_q // H_kv
+    q = rng.normal(size=(H_q, 1, d))
+    k = rng.normal(size=(H_kv, P + 1, d))
+    res = O.select_chunk(q, k, P, 1, B)
+    for g in range(H_kv):
+        qg = torch.as_tensor(q[g * G:(g + 1) * G, 0])                  # [G, d]
+        kg = torch.as_tensor(k[g, :P])                                 # [P, d]
+        cos = F.cosine_similarity(qg[:, None, :], kg[None, :, :], dim=-1)
+        expect = cos.mean(0).numpy()
+        np.testing.assert_allclose(res["score"][g], expect, rtol=1e-12, atol=1e-14)
+        top = np.sort(np.argsort(-expect, kind="stable")[:B])
+        assert res["idx"][g].tolist() == top.tolist()
+    k2 = k.copy()
+    k2[:, :P] *= rng.uniform(0.1, 10.0, size=(H_kv, P, 1))
+    res2 = O.select_chunk(q, k2, P, 1, B)
+    np.testing.assert_allclose(res2["score"], res["score"], rtol=1e-12, atol=1e-14)
+
+
 def _sdpa_masked(q, k, v, mask_of_head):
     """Library attention (fp64 torch SDPA) per query head with an explicit bool mask."""
     H_q, H_kv = q.shape[0], k.shape[0]
@@ -338,7 +363,8 @@ ALL_PINS = [pin_query_cosine_closed_form, pin_subselect_brute_force, pin_query_s
             pin_scoring_closed_forms, pin_key_scale_and_permutation, pin_top_budget_brute_force,
             pin_worked_example, pin_attention_vs_sdpa, pin_full_budget_is_full_causal,
             pin_gqa_is_independent_mqa, pin_prefill_full_budget_is_causal,
-            pin_prefill_zero_budget_is_block_causal, pin_prefill_is_causal_over_chunks]
+            pin_prefill_zero_budget_is_block_causal, pin_prefill_is_causal_over_chunks,
+            pin_decode_is_mean_cosine]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
