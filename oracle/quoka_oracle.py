@@ -37,6 +37,11 @@ set, so the oracle follows the method's steps in the pages' order:
 7. whole-prompt chunked prefill (Figure 1(a): a prompt cut into chunks, each chunk
    sub-selecting the cache that the chunks before it wrote): chunk c has prefix
    P = c * C, selects over rows 0 .. P-1 with that chunk's budget, and attends.
+8. per-query sparse attention (QUILT page, summary: each query has its own selected
+   key-value entries, and nearby queries share many of them): query t of head h
+   attends to exactly its own set of key positions, softmax(q k^T / sqrt(d)) v over
+   that set.  This is what shared-query execution must reproduce, whatever grouping
+   and union loading it uses.
 
 Readings where the pages are silent (each is listed with its reason in the design
 notes of the repository): the budget B counts prefix keys only and the chunk's own
@@ -58,7 +63,7 @@ import numpy as np
 __all__ = [
     "unit_rows", "mean_query", "query_cosines", "subselect_queries", "pooled_key_scores",
     "top_budget", "select_chunk", "attend_chunk", "select_batch", "attend_batch",
-    "prefill_prompt",
+    "prefill_prompt", "attend_per_query",
 ]
 
 
@@ -277,3 +282,29 @@ def prefill_prompt(q_prompt, k_prompt, v_prompt, chunk: int, nq: int,
         out[:, P:P + C] = attend_chunk(qc, k[:, :P + C], v[:, :P + C], P, sel["idx"])
         idx.append(sel["idx"])
     return {"out": out, "idx": idx}
+
+
+def attend_per_query(q, k, v, sel) -> np.ndarray:
+    """Step 8: every query row over its own selected keys.
+
+    q [H_q, T, d]; k, v [H_kv, N, d] (rows of one sequence); sel int [H_q, T, S]: the
+    key positions query (h, t) attends to, padded with -1 (duplicates count once).
+    Query head h reads KV head h // G.  Returns O [H_q, T, d].
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    sel = np.asarray(sel, dtype=np.int64)
+    H_q, T, d = q.shape
+    G = H_q // k.shape[0]
+    scale = 1.0 / np.sqrt(d)
+    out = np.zeros((H_q, T, d))
+    for h in range(H_q):
+        g = h // G
+        for t in range(T):
+            keys = np.unique(sel[h, t][sel[h, t] >= 0])
+            assert keys.size > 0, "every query needs at least one key"
+            logits = (k[g, keys] @ q[h, t]) * scale
+            p = np.exp(logits - logits.max())
+            out[h, t] = (p @ v[g, keys]) / p.sum()
+    return out

@@ -215,3 +215,28 @@ def generate(w: Workload) -> Tensors:
     dt = w.torch_dtype
     return Tensors(q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous(),
                    tuple(kv_off))
+
+
+def per_query_selection(seed: int, h_q: int, n_queries: int, n_keys: int, s: int,
+                        group: int = 16, shared: float = 0.75) -> torch.Tensor:
+    """Per-query key sets with locality, the input of shared-query execution (QUILT page:
+    nearby queries select many of the same key-value entries).  Per query head, every run
+    of `group` consecutive queries draws one base set of s keys; each query keeps
+    round(shared * s) of them and draws the rest on its own, without repeats.  Returns
+    int32 [h_q, n_queries, s], each row ascending."""
+    if s > n_keys:
+        raise ValueError("s must not exceed n_keys")
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    keep = int(round(shared * s))
+    out = torch.empty(h_q, n_queries, s, dtype=torch.int32)
+    for h in range(h_q):
+        for t0 in range(0, n_queries, group):
+            base = torch.randperm(n_keys, generator=g)[:s]
+            for t in range(t0, min(n_queries, t0 + group)):
+                mine = base[torch.randperm(s, generator=g)[:keep]]
+                taken = torch.zeros(n_keys, dtype=torch.bool)
+                taken[mine] = True
+                rest = torch.randperm(n_keys, generator=g)
+                rest = rest[~taken[rest]][:s - keep]
+                out[h, t] = torch.sort(torch.cat([mine, rest])).values.to(torch.int32)
+    return out

@@ -285,6 +285,40 @@ def pin_decode_is_mean_cosine(seed=14):
     np.testing.assert_allclose(res2["score"], res["score"], rtol=1e-12, atol=1e-14)
 
 
+def pin_per_query_vs_sdpa(seed=15):
+    """Per-query selections (the QUILT setting): each query over exactly its own keys
+    equals torch SDPA with a per-query boolean mask; a shared set reduces to the chunk
+    attention of step 6 with that set and no chunk keys visible."""
+    rng = np.random.default_rng(seed)
+    H_q, H_kv, T, N, d, S = 4, 2, 6, 30, 8, 5
+    G = H_q // H_kv
+    q = rng.normal(size=(H_q, T, d))
+    k = rng.normal(size=(H_kv, N, d))
+    v = rng.normal(size=(H_kv, N, d))
+    sel = rng.integers(0, N, size=(H_q, T, S))
+    sel[0, 0, 2:] = -1                                  # padding
+    sel[1, 3, 1] = sel[1, 3, 0]                         # a duplicate counts once
+    o = O.attend_per_query(q, k, v, sel)
+    for h in range(H_q):
+        mask = torch.zeros(T, N, dtype=torch.bool)
+        for t in range(T):
+            for j in sel[h, t]:
+                if j >= 0:
+                    mask[t, j] = True
+        ref = F.scaled_dot_product_attention(
+            torch.as_tensor(q[h])[None, None], torch.as_tensor(k[h // G])[None, None],
+            torch.as_tensor(v[h // G])[None, None], attn_mask=mask)[0, 0].numpy()
+        np.testing.assert_allclose(o[h], ref, rtol=1e-12, atol=1e-13)
+    shared = np.sort(rng.choice(N - T, size=S, replace=False))
+    sel2 = np.broadcast_to(shared, (H_q, 1, S)).copy()
+    o2 = O.attend_per_query(q[:, :1], k, v, sel2)
+    # step 6 with the prefix ending at the largest shared key: chunk position 0 attends to
+    # the other shared keys (selected) plus its own row P, i.e. exactly the shared set
+    P = int(shared[-1])
+    o6 = O.attend_chunk(q[:, :1], k, v, P, [shared[:-1]] * H_kv)
+    np.testing.assert_allclose(o2, o6, rtol=1e-12, atol=1e-13)
+
+
 def _sdpa_masked(q, k, v, mask_of_head):
     """Library attention (fp64 torch SDPA) per query head with an explicit bool mask."""
     H_q, H_kv = q.shape[0], k.shape[0]
@@ -364,7 +398,7 @@ ALL_PINS = [pin_query_cosine_closed_form, pin_subselect_brute_force, pin_query_s
             pin_worked_example, pin_attention_vs_sdpa, pin_full_budget_is_full_causal,
             pin_gqa_is_independent_mqa, pin_prefill_full_budget_is_causal,
             pin_prefill_zero_budget_is_block_causal, pin_prefill_is_causal_over_chunks,
-            pin_decode_is_mean_cosine]
+            pin_decode_is_mean_cosine, pin_per_query_vs_sdpa]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
