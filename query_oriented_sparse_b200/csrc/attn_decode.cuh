@@ -260,7 +260,7 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 #pragma unroll
     for (int e = 0; e < EPL; ++e) wout[r * D + lane * EPL + e] = acc[r][e];
   __syncthreads();
-  float* dst = part + ((size_t)((b * h_kv + g) * nsplit_ws + s) * R) * Cfg::PD;
+  float* dst = part + (((size_t)(b * h_kv + g) * nsplit_ws + s) * R) * Cfg::PD;
   for (int e = threadIdx.x; e < R * D; e += blockDim.x) {
     const int r = e / D, d = e - r * D;
     float M = -INFINITY;
