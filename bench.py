@@ -597,6 +597,36 @@ def dense_reference_ms(q, k_new, v_new, steps, flush):
         return None
 
 
+def oracle_prompt_sample(w, t, rows: int = 64):
+    """Times the fp64 oracle on a bounded sample of the whole-prompt prefill: the last
+    chunk's selection for KV head 0 plus attention for `rows` sampled query rows of that
+    chunk; extrapolates selection by prefix length over the chunks that select (times the
+    KV heads) and attention by keys per query row over every row of the prompt."""
+    from oracle import quoka_oracle as O
+    C, n, G = w.chunk, w.prompt_chunks, w.group
+    budgets = w.budgets_of_chunks()
+    c = n - 1
+    P = c * C
+    q = t.q[0, 0:G, P:P + C].double().numpy()
+    k = t.k_cache[0:1, :P + C].double().numpy()
+    v = t.v_cache[0:1, :P + C].double().numpy()
+    t0 = time.perf_counter()
+    res = O.select_chunk(q, k[:, :P], P, w.nq, budgets[c])
+    t_sel = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    rr = [(int(rng.integers(G)), int(rng.integers(C))) for _ in range(rows)]
+    t0 = time.perf_counter()
+    O.attend_chunk(q, k, v, P, res["idx"], rows=rr)
+    t_att = time.perf_counter() - t0
+    sel_prefix = sum(cc * C for cc in range(1, n) if budgets[cc] > 0)
+    keys_sample = sum(min(budgets[c], P) + tt + 1 for _, tt in rr) / rows
+    keys_total = w.h_q * sum(C * min(budgets[cc], cc * C) + C * (C + 1) / 2 for cc in range(n))
+    est = t_sel * w.h_kv * sel_prefix / P + t_att / rows / keys_sample * keys_total
+    return {"ttft_s": est, "sample": f"chunk {c}'s selection for KV head 0 (P={P}) + attention "
+                                     f"for {rows} sampled query rows of that chunk; extrapolated "
+                                     f"to {n} chunks x {w.h_kv} KV heads x {w.h_q * C * n} query rows"}
+
+
 def run_prefill(args, w):
     from query_oriented_sparse_b200 import binding as Bd
 
@@ -645,6 +675,64 @@ def run_prefill(args, w):
     roof_ms = sum(rl.values()) / 1e3
     dense_ms = dense_reference_ms(q, kn, vn, max(1, min(args.steps, 3)), flush)
     n_sel = sum(1 for c, bgt in enumerate(budgets) if c > 0 and bgt > 0)
+    att_tflops = st["attn"]["flops"] / (ttft / 1e3) / 1e12
+
+    # End to end: the prompt lives in pinned host memory and goes through quoka_step chunk
+    # by chunk, as a server streams it: chunk c+1's inputs are uploaded on one copy stream
+    # and chunk c's output read back on another while chunk c computes (inputs and outputs
+    # double-buffered).  Timed from the first upload to the last read-back.
+    n, C = w.prompt_chunks, w.chunk
+    q_h, kn_h, vn_h = q.cpu().pin_memory(), kn.cpu().pin_memory(), vn.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    qd = [torch.empty_like(q[0]) for _ in range(2)]
+    knd = [torch.empty_like(kn[0]) for _ in range(2)]
+    vnd = [torch.empty_like(vn[0]) for _ in range(2)]
+    od = [torch.empty_like(out[0]) for _ in range(2)]
+    sws = torch.empty(Bd.step_workspace_size(shape, (n - 1) * C, w.nq, b_max), dtype=torch.uint8,
+                      device=dev)
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_prompt():
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for c in range(n):
+            bb = c & 1
+            with torch.cuda.stream(s_in):
+                if c >= 2:
+                    s_in.wait_event(ev_cmp[bb])
+                if c == 0:
+                    t0.record(s_in)
+                qd[bb].copy_(q_h[c], non_blocking=True)
+                knd[bb].copy_(kn_h[c], non_blocking=True)
+                vnd[bb].copy_(vn_h[c], non_blocking=True)
+                ev_in[bb].record(s_in)
+            stream.wait_event(ev_in[bb])
+            if c >= 2:
+                stream.wait_event(ev_out[bb])
+            Bd.quoka_step(qd[bb], knd[bb], vnd[bb], k, v, t.kv_off, [c * C] * w.batch, w.nq,
+                          [budgets[c]] * w.batch, idx, out=od[bb], workspace=sws)
+            ev_cmp[bb].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[bb])
+                out_h[c].copy_(od[bb], non_blocking=True)
+                ev_out[bb].record(s_out)
+        t1.record(s_out)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
+
+    e2e_ms = []
+    for i in range(1 + args.steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        e = e2e_prompt()
+        if i > 0:
+            e2e_ms.append(e)
+    assert Bd.device_error() == 0
+    assert torch.equal(out_h, out.cpu()), "the streamed prompt differs from the prefill call"
+    e2e_value = statistics.median(e2e_ms)
+    cpu = oracle_prompt_sample(w, t) if not args.no_cpu_baseline else None
     line = {
         "metric": PREFILL_METRIC, "value": ttft, "unit": "ms", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ttft,
@@ -656,13 +744,26 @@ def run_prefill(args, w):
                    "budget_per_chunk": "c * chunk / 8",
                    "l2": "256 MB flush before every timed prompt"},
         "tokens_per_s": tokens / (ttft / 1e3),
+        "e2e": {"value": e2e_value, "unit": "ms",
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (q_h, kn_h, vn_h)),
+                "d2h_bytes_per_step": out_h.numel() * out_h.element_size()},
         "gpu_launches": (2 * w.prompt_chunks + 3 * n_sel) * args.steps,
+        "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16_tflops"],
+                     "traffic": None,
+                     "kernel": "attn_tc2_kernel over the prompt's chunks, timed as the whole "
+                               "prefill call (selection included, so this understates the "
+                               "kernel's own rate)",
+                     "peak_source": f"{peak_src} bf16 dense (burst)"},
         "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ttft,
                           "peak_source": f"{peak_src} bf16 dense (burst) and HBM copy"},
         "dense_sdpa_ms": dense_ms,
         "ttft_reduction_vs_dense": (dense_ms / ttft) if dense_ms else None,
         "clocks": clk.summary(),
     }
+    if cpu is not None:
+        line["cpu_baseline"] = {"value": cpu["ttft_s"] * 1e3, "unit": "ms", "cores": blas_threads(),
+                                "kind": "oracle", "sample": cpu["sample"]}
     print(json.dumps(line), flush=True)
     return 0
 

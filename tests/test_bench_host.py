@@ -82,3 +82,19 @@ def test_attn_traffic_is_pinned_to_workload():
     assert bench.attn_traffic(W.WORKLOADS["gqa_8k"]) is None
     t = bench.attn_traffic(W.WORKLOADS["ctx_128k"])
     assert t is None or abs(t - 139.38e6) < 1e5
+
+
+def test_oracle_prompt_sample_extrapolates():
+    """The prefill line's CPU baseline: a bounded oracle sample scaled to the prompt,
+    within a small factor of running the whole oracle loop on a small prompt."""
+    import time
+    from oracle import quoka_oracle as O
+    w = W.custom("pp", h_q=8, h_kv=2, head_dim=64, chunk=64, prefix=0, nq=8, budget=64, seed=1,
+                 prompt_chunks=5, chunk_budget=(0, 8, 16, 24, 32))
+    t = W.generate(w)
+    r = bench.oracle_prompt_sample(w, t, rows=32)
+    t0 = time.perf_counter()
+    O.prefill_prompt(t.q[0], t.k_cache, t.v_cache, 64, 8, w.budgets_of_chunks())
+    full = time.perf_counter() - t0
+    assert 0.2 * full < r["ttft_s"] < 5.0 * full
+    assert "chunk 4" in r["sample"]
