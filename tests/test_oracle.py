@@ -578,10 +578,39 @@ def _mut_prefill_budget_shift(mp):
                orig(q, k, v, chunk, nq, [budgets[0]] + list(budgets[:-1])))
 
 
+def _per_query_variant(dedupe: bool, drop_padding: bool):
+    def bad(q, k, v, sel):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        sel = np.asarray(sel, dtype=np.int64)
+        H_q, T, d = q.shape
+        G = H_q // k.shape[0]
+        out = np.zeros((H_q, T, d))
+        for h in range(H_q):
+            for t in range(T):
+                keys = sel[h, t][sel[h, t] >= 0] if drop_padding else sel[h, t]
+                keys = np.unique(keys) if dedupe else keys
+                logits = (k[h // G, keys] @ q[h, t]) / np.sqrt(d)
+                p = np.exp(logits - logits.max())
+                out[h, t] = (p @ v[h // G, keys]) / p.sum()
+        return out
+    return bad
+
+
+def _mut_per_query_counts_duplicates(mp):
+    """A key listed twice in a query's set weighs twice."""
+    mp.setattr(O, "attend_per_query", _per_query_variant(dedupe=False, drop_padding=True))
+
+
+def _mut_per_query_reads_padding(mp):
+    """Padding (-1) read as the last key row."""
+    mp.setattr(O, "attend_per_query", _per_query_variant(dedupe=True, drop_padding=False))
+
+
 MUTANTS = [_mut_most_similar, _mut_raw_mean, _mut_max_over_group, _mut_mean_then_max,
            _mut_no_key_norm, _mut_ties_high_index, _mut_no_softmax_scale,
            _mut_causal_excludes_self, _mut_prefill_own_chunk_candidates,
-           _mut_prefill_budget_shift]
+           _mut_prefill_budget_shift, _mut_per_query_counts_duplicates,
+           _mut_per_query_reads_padding]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)
