@@ -1,7 +1,8 @@
 """The C ABI library: it loads, exports every symbol include/quoka.h declares, and its
 host-side validation rejects bad calls with the documented status before launching
-anything.  The fake-pointer cases run only where no GPU is present (on a GPU machine the
-same rejections are exercised with real buffers in test_kernels.py)."""
+anything.  The fake-pointer cases run only where no GPU is present (with a GPU the
+same rejections are exercised with real buffers in test_kernels.py, test_prefill.py and
+test_step.py)."""
 import ctypes
 import os
 import re
