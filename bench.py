@@ -370,9 +370,9 @@ def run_ours(args, w):
     launch_mode = "eager"
     if not args.eager:
         g_sel, g_att = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_sel):
+        with torch.cuda.graph(g_sel, capture_error_mode="thread_local"):
             select()
-        with torch.cuda.graph(g_att):
+        with torch.cuda.graph(g_att, capture_error_mode="thread_local"):
             attend()
         select, attend = g_sel.replay, g_att.replay
         launch_mode = "CUDA graph per call, captured once and replayed every step"
@@ -447,7 +447,7 @@ def run_ours(args, w):
     if not args.eager:
         g_step = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
         for b in range(2):
-            with torch.cuda.graph(g_step[b]):
+            with torch.cuda.graph(g_step[b], capture_error_mode="thread_local"):
                 step_on[b]()
         step_on = [g.replay for g in g_step]
 
