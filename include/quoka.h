@@ -164,6 +164,37 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk,
 size_t sparse_chunk_attn_workspace_size(const quoka_shape* shape, int b_max);
 
 /*
+ * sparse_perq_attn - attention where every query has its own selected keys, computed
+ * with shared loading (QUILT page, summary: nearby queries are grouped, the key-value
+ * entries they selected are loaded once and reused for all of them).
+ *
+ * Query t of head h of sequence b (KV head g = h / G) attends to exactly the positions
+ * { sel[b, h, t, i] : i < S, sel[b, h, t, i] >= 0 } of its sequence's cache rows
+ * (duplicates count once), out = softmax(q . k^T / sqrt(head_dim)) . v, fp32 softmax,
+ * stored in `dtype`; a query whose set is empty gets zeros.  Causality is the caller's:
+ * any position of the sequence may be listed.  Tiles of the G heads x (16 / G)
+ * consecutive positions of a KV head load the union of their sets once.
+ *
+ *   q_chunk     device, [batch, h_q, chunk, head_dim]
+ *   k_cache, v_cache  device, [h_kv, kv_off[batch], head_dim]
+ *   kv_off      host, batch + 1 nondecreasing offsets, every sequence 1 .. 262144 rows
+ *   sel         device int32 [batch, h_q, chunk, S]: positions relative to the sequence's
+ *               first row, or -1; a position past the sequence sets the device error
+ *               word and is ignored
+ *   S           entries per query, 1 .. 2^20
+ *   out         device, [batch, h_q, chunk, head_dim]; must not alias an input
+ *   workspace   device scratch of sparse_perq_attn_workspace_size(shape, S) bytes
+ * Limits: h_q / h_kv <= 16.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+quoka_status sparse_perq_attn(const quoka_shape* shape, const void* q_chunk,
+                              const void* k_cache, const void* v_cache,
+                              const int64_t* kv_off, const int32_t* sel, int S, void* out,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device scratch sparse_perq_attn() needs (0 if the arguments are invalid). */
+size_t sparse_perq_attn_workspace_size(const quoka_shape* shape, int S);
+
+/*
  * quoka_step - one step of a chunked prefill or of decode, the way a serving loop runs
  * it: the chunk's new K/V rows go into the cache inside the call, then quoka_select and
  * sparse_chunk_attn run as described above (QUOKA page, Figure 1(a): each chunk sub-

@@ -48,6 +48,9 @@ SIGNATURES = {
     "quoka_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "quoka_select_noalloc": (ctypes.c_int, [_SHAPE_P, _P, _P, _I64P, _I32P, ctypes.c_int, _I32P,
                                             ctypes.c_int, _P, _P, _P]),
+    "sparse_perq_attn": (ctypes.c_int, [_SHAPE_P, _P, _P, _P, _I64P, _P, ctypes.c_int, _P, _P,
+                                        ctypes.c_size_t, _P]),
+    "sparse_perq_attn_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int]),
     "quoka_step": (ctypes.c_int, [_SHAPE_P, _P, _P, _P, _P, _P, _I64P, _I32P, ctypes.c_int,
                                   _I32P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "quoka_step_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int, ctypes.c_int,
@@ -207,6 +210,30 @@ def sparse_chunk_attn(q_chunk: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
         ctypes.byref(shape), _ptr(q_chunk), _ptr(k_cache), _ptr(v_cache), _host_i64(kv_off),
         _host_i32(prefix_len), _host_i32(budget), _ptr(idx), b_max, _ptr(out), _ptr(workspace),
         ws_bytes, ctypes.c_void_p(_stream(stream))))
+    return out
+
+
+def perq_workspace_size(shape: QuokaShape, S: int) -> int:
+    return int(lib().sparse_perq_attn_workspace_size(ctypes.byref(shape), int(S)))
+
+
+def sparse_perq_attn(q_chunk: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                     kv_off: Sequence[int], sel: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Every query over its own key set, sel int32 [batch, h_q, C, S] (-1 = none);
+    returns out [batch, h_q, C, d]."""
+    shape = shape_of(q_chunk, k_cache)
+    if out is None:
+        out = torch.empty_like(q_chunk)
+    S = int(sel.shape[-1])
+    if workspace is None:
+        n = perq_workspace_size(shape, S)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q_chunk.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().sparse_perq_attn(
+        ctypes.byref(shape), _ptr(q_chunk), _ptr(k_cache), _ptr(v_cache), _host_i64(kv_off),
+        _ptr(sel), S, _ptr(out), _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(stream))))
     return out
 
 

@@ -21,6 +21,7 @@
 #include "compact.cuh"
 #include "attn_decode.cuh"
 #include "select_decode.cuh"
+#include "attn_perq.cuh"
 
 using namespace quoka;
 
@@ -537,6 +538,81 @@ quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, con
   return QUOKA_OK;
 }
 
+// ---- per-query selections (shared loading per tile) --------------------------------
+struct PerqPlan {
+  int TQ, R, ntiles, split, nsplit;
+  size_t uni, memb, ucount, part, total;
+};
+
+PerqPlan perq_plan(const Dims& d, int S) {
+  PerqPlan p;
+  p.TQ = std::max(1, PQ_MAX_ROWS / d.G);
+  p.R = 1;
+  while (p.R < d.G * p.TQ) p.R *= 2;
+  p.ntiles = (d.C + p.TQ - 1) / p.TQ;
+  // the union of a tile is at most PQ_MAX_ROWS * S keys: up to eight splits of it
+  const int nw = d.dt == QUOKA_F32 && d.D == 128 ? 2 : 4;     // AdcCfg<T, D>::NW
+  const long long ub = (long long)PQ_MAX_ROWS * S;
+  long long split = (ub + 7) / 8;
+  split = (split + 32 * nw - 1) / (32 * nw) * (32 * nw);
+  p.split = (int)std::min<long long>(std::max<long long>(split, ADC_MIN_SPLIT), ADC_MAX_SPLIT);
+  p.nsplit = (int)((ub + p.split - 1) / p.split);
+  const size_t nbt = (size_t)d.batch * d.h_kv * p.ntiles;
+  size_t off = 0;
+  p.uni = off;
+  off = align_up(off + nbt * ub * 4, 256);
+  p.memb = off;
+  off = align_up(off + nbt * ub * 4, 256);
+  p.ucount = off;
+  off = align_up(off + nbt * 4, 256);
+  p.part = off;
+  off = align_up(off + nbt * p.nsplit * p.R * (size_t)(d.D + 4) * 4, 256);
+  p.total = off;
+  return p;
+}
+
+template <typename T, int D, int R>
+quoka_status launch_perq_r(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                           const void* k, const void* v, const int32_t* sel, int S, void* out,
+                           unsigned char* ws, const PerqPlan& pl, cudaStream_t st) {
+  using Cfg = AdcCfg<T, D>;
+  auto* uni = reinterpret_cast<int32_t*>(ws + pl.uni);
+  auto* memb = reinterpret_cast<uint32_t*>(ws + pl.memb);
+  auto* ucount = reinterpret_cast<int32_t*>(ws + pl.ucount);
+  auto* part = reinterpret_cast<float*>(ws + pl.part);
+  cudaError_t e;
+  const int usmem = 2 * PQ_MAX_WORDS * 4;
+  if ((e = ensure_smem(perq_union_kernel, usmem)) != cudaSuccess) return cuda_fail(e, "perq_union smem");
+  perq_union_kernel<<<dim3(pl.ntiles, d.h_kv, d.batch), PQ_UNION_THREADS, usmem, st>>>(
+      sel, tab, d.h_q, d.h_kv, d.C, S, pl.TQ, uni, memb, ucount);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_union launch");
+  const int smem = adc_smem_bytes<T, D, R>();
+  if ((e = ensure_smem(perq_attn_kernel<T, D, R>, smem)) != cudaSuccess) return cuda_fail(e, "perq_attn smem");
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  perq_attn_kernel<T, D, R><<<dim3(pl.nsplit, pl.ntiles, d.batch * d.h_kv), Cfg::THREADS, smem, st>>>(
+      reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(k), reinterpret_cast<const T*>(v),
+      rows, tab, d.h_q, d.h_kv, d.C, S, pl.TQ, uni, memb, ucount, pl.split, pl.nsplit, scale_log2,
+      part);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_attn launch");
+  perq_combine_kernel<T, D, R><<<dim3(pl.ntiles, d.batch * d.h_kv), 128, 0, st>>>(
+      part, ucount, d.h_q, d.h_kv, d.C, pl.TQ, pl.split, pl.nsplit, reinterpret_cast<T*>(out));
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_combine launch");
+  return QUOKA_OK;
+}
+
+template <typename T, int D>
+quoka_status launch_perq(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                         const void* k, const void* v, const int32_t* sel, int S, void* out,
+                         unsigned char* ws, const PerqPlan& pl, cudaStream_t st) {
+  switch (pl.R) {
+    case 1: return launch_perq_r<T, D, 1>(d, tab, rows, q, k, v, sel, S, out, ws, pl, st);
+    case 2: return launch_perq_r<T, D, 2>(d, tab, rows, q, k, v, sel, S, out, ws, pl, st);
+    case 4: return launch_perq_r<T, D, 4>(d, tab, rows, q, k, v, sel, S, out, ws, pl, st);
+    case 8: return launch_perq_r<T, D, 8>(d, tab, rows, q, k, v, sel, S, out, ws, pl, st);
+    default: return launch_perq_r<T, D, 16>(d, tab, rows, q, k, v, sel, S, out, ws, pl, st);
+  }
+}
+
 // One step with the append: select over each sequence's prefix (when any key is to be
 // kept), then attend, the chunk's new K/V rows going into the cache on the way (fused
 // with the compaction where there is one).
@@ -676,6 +752,56 @@ quoka_status sparse_chunk_attn(const quoka_shape* shape, const void* q_chunk, co
   }
   return d.D == 64 ? launch_attn<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st)
                    : launch_attn<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, v_cache, idx, b_max, out, ws, st);
+}
+
+size_t sparse_perq_attn_workspace_size(const quoka_shape* shape, int S) {
+  Dims d;
+  if (check_shape(shape, &d) != QUOKA_OK || S < 1 || d.G > PQ_MAX_ROWS) return 0;
+  return perq_plan(d, S).total;
+}
+
+quoka_status sparse_perq_attn(const quoka_shape* shape, const void* q_chunk, const void* k_cache,
+                              const void* v_cache, const int64_t* kv_off, const int32_t* sel,
+                              int S, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (d.G > PQ_MAX_ROWS)
+    return fail(QUOKA_ERR_UNSUPPORTED, "per-query attention takes at most %d query heads per KV head (got %d)",
+                PQ_MAX_ROWS, d.G);
+  if (!q_chunk || !k_cache || !v_cache || !kv_off || !sel || !out)
+    return fail(QUOKA_ERR_INVALID_ARG, "q_chunk, k_cache, v_cache, kv_off, sel and out must be non-NULL");
+  if (!aligned(q_chunk, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(sel, 16) ||
+      !aligned(out, 16))
+    return fail(QUOKA_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (out == q_chunk || out == k_cache || out == v_cache)
+    return fail(QUOKA_ERR_INVALID_ARG, "out must not alias an input");
+  if (S < 1 || S > (1 << 20)) return fail(QUOKA_ERR_INVALID_ARG, "S must be in [1, 2^20] (got %d)", S);
+  if (kv_off[0] < 0) return fail(QUOKA_ERR_INVALID_ARG, "kv_off[0] must be >= 0");
+  SeqTable tab;
+  tab.batch = d.batch;
+  tab.max_prefix = 0;
+  for (int b = 0; b <= d.batch; ++b) tab.kv_off[b] = kv_off[b];
+  for (int b = 0; b < QUOKA_MAX_BATCH; ++b) { tab.prefix[b] = 0; tab.nsel[b] = 0; }
+  for (int b = 0; b < d.batch; ++b) {
+    const long long n = kv_off[b + 1] - kv_off[b];
+    if (n < 1) return fail(QUOKA_ERR_INVALID_ARG, "sequence %d owns no cache rows", b);
+    if (n > (long long)PQ_MAX_WORDS * 32)
+      return fail(QUOKA_ERR_UNSUPPORTED, "sequence %d owns %lld rows; per-query attention takes at most %d",
+                  b, n, PQ_MAX_WORDS * 32);
+  }
+  const PerqPlan pl = perq_plan(d, S);
+  if (!workspace) return fail(QUOKA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", pl.total);
+  if (!aligned(workspace, 256)) return fail(QUOKA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < pl.total) return fail(QUOKA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, pl.total);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* ws = reinterpret_cast<unsigned char*>(workspace);
+  const long long rows = kv_off[d.batch];
+  if (d.dt == QUOKA_F32)
+    return d.D == 64 ? launch_perq<float, 64>(d, tab, rows, q_chunk, k_cache, v_cache, sel, S, out, ws, pl, st)
+                     : launch_perq<float, 128>(d, tab, rows, q_chunk, k_cache, v_cache, sel, S, out, ws, pl, st);
+  return d.D == 64 ? launch_perq<__nv_bfloat16, 64>(d, tab, rows, q_chunk, k_cache, v_cache, sel, S, out, ws, pl, st)
+                   : launch_perq<__nv_bfloat16, 128>(d, tab, rows, q_chunk, k_cache, v_cache, sel, S, out, ws, pl, st);
 }
 
 size_t quoka_step_workspace_size(const quoka_shape* shape, int max_prefix, int nq, int b_max) {
