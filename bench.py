@@ -768,6 +768,100 @@ def run_prefill(args, w):
     return 0
 
 
+# --------------------------------------------------------------------------------------
+# per-query selections with shared loading
+# --------------------------------------------------------------------------------------
+
+PERQ_METRIC = "per-query sparse attention tokens/s (each query its own key set), 1 B200"
+PERQ_S = 512               # keys per query
+PERQ_GROUP = 16            # consecutive queries drawing from one base set
+
+
+def perq_union_rows(sel, h_kv, tq):
+    """Union size of every tile (G heads x tq positions of a KV head) and the rows the
+    tiles would load without sharing; sel int32 [h_q, C, S] on the CPU."""
+    h_q, C, S = sel.shape
+    G = h_q // h_kv
+    nt = C // tq
+    x = sel[:, :nt * tq].reshape(h_kv, G, nt, tq, S).permute(0, 2, 1, 3, 4).reshape(h_kv * nt, -1)
+    x = torch.sort(x.long(), dim=1).values
+    distinct = 1 + (x[:, 1:] != x[:, :-1]).sum(dim=1)
+    return int(distinct.sum()), int(x.shape[0] * x.shape[1])
+
+
+def run_perq(args):
+    from query_oriented_sparse_b200 import binding as Bd
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--perq runs on one GPU")
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks, peak_src = load_peaks()
+    w = W.WORKLOADS["ctx_128k"]
+    t = W.generate(w)
+    n_rows = t.kv_off[1]
+    sel_h = W.per_query_selection_large(7, w.h_q, w.chunk, n_rows, PERQ_S, group=PERQ_GROUP)
+    tq = max(1, 16 // w.group)
+    union_rows, flat_rows = perq_union_rows(sel_h, w.h_kv, tq)
+    q, k, v = t.q.to(dev), t.k_cache.to(dev), t.v_cache.to(dev)
+    sel = sel_h[None].contiguous().to(dev)
+    shape = Bd.shape_of(q, k)
+    ws = torch.empty(Bd.perq_workspace_size(shape, PERQ_S), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def call():
+        Bd.sparse_perq_attn(q, k, v, t.kv_off, sel, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    assert Bd.device_error() == 0
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        call()
+    stream = torch.cuda.current_stream()
+    ms = []
+    with ClockSampler(0) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+    assert Bd.device_error() == 0
+    t_ms = statistics.median(ms)
+    tokens = w.chunk
+    row = w.head_dim * 2
+    # compulsory bytes: the index sets, Q and O, and each tile's union of K and V rows once
+    by = sel.numel() * 4 + 2 * q.numel() * 2 + 2 * union_rows * row
+    fl = 4.0 * w.head_dim * w.h_q * w.chunk * PERQ_S
+    gbs = by / (t_ms / 1e3) / 1e9
+    line = {
+        "metric": PERQ_METRIC, "value": tokens / (t_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "perq_128k", "chunk": w.chunk, "cache_rows": n_rows,
+                   "h_q": w.h_q, "h_kv": w.h_kv, "head_dim": w.head_dim, "keys_per_query": PERQ_S,
+                   "locality_group": PERQ_GROUP, "tile_rows": w.group * tq,
+                   "l2": "256 MB flush before every timed call",
+                   "launch": "CUDA graph, captured once and replayed every step"},
+        "gpu_launches": 3 * args.steps,
+        "union_rows": union_rows, "rows_without_sharing": flat_rows,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "perq_union_kernel + perq_attn_kernel + combine, timed as the call",
+                     "peak_source": f"{peak_src} HBM copy", "flops": fl},
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -780,7 +874,13 @@ def main():
                     help="launch every call from the host each step instead of replaying graphs")
     ap.add_argument("--prefill", nargs="?", const="prompt_128k", choices=sorted(W.PROMPTS),
                     help="time a whole prompt through the prefill call (time to first token)")
+    ap.add_argument("--perq", action="store_true",
+                    help="time per-query sparse attention with shared loading")
     args = ap.parse_args()
+    if args.perq:
+        if args.impl != "ours":
+            raise SystemExit("--perq has no reference arm")
+        return run_perq(args)
     if args.prefill:
         if args.impl != "ours":
             raise SystemExit("--prefill has no reference arm")

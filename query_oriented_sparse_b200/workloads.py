@@ -240,3 +240,23 @@ def per_query_selection(seed: int, h_q: int, n_queries: int, n_keys: int, s: int
                 rest = rest[~taken[rest]][:s - keep]
                 out[h, t] = torch.sort(torch.cat([mine, rest])).values.to(torch.int32)
     return out
+
+
+def per_query_selection_large(seed: int, h_q: int, n_queries: int, n_keys: int, s: int,
+                              group: int = 16, shared: float = 0.75) -> torch.Tensor:
+    """per_query_selection for large sizes, vectorised per head: every run of `group`
+    consecutive queries draws one base set; each entry of a query's set is the base
+    set's entry at that slot with probability `shared`, else a draw of its own.  Draws
+    are with replacement, so a set may hold a position twice (the attention counts it
+    once).  Returns int32 [h_q, n_queries, s], rows ascending."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    ngroups = (n_queries + group - 1) // group
+    gid = torch.arange(n_queries) // group
+    out = torch.empty(h_q, n_queries, s, dtype=torch.int32)
+    for h in range(h_q):
+        base = torch.randint(0, n_keys, (ngroups, s), generator=g)
+        own = torch.randint(0, n_keys, (n_queries, s), generator=g)
+        take = torch.rand(n_queries, s, generator=g) < shared
+        rows = torch.where(take, base[gid], own)
+        out[h] = torch.sort(rows, dim=1).values.to(torch.int32)
+    return out

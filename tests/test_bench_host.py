@@ -98,3 +98,11 @@ def test_oracle_prompt_sample_extrapolates():
     full = time.perf_counter() - t0
     assert 0.2 * full < r["ttft_s"] < 5.0 * full
     assert "chunk 4" in r["sample"]
+
+
+def test_perq_union_rows_counts_distinct_per_tile():
+    sel = W.per_query_selection_large(1, 8, 64, 3000, 32, group=16)
+    u, flat = bench.perq_union_rows(sel, 2, 4)
+    ref = sum(len(set(sel[4 * g:4 * g + 4, t0:t0 + 4].flatten().tolist()))
+              for g in range(2) for t0 in range(0, 64, 4))
+    assert u == ref and flat == 2 * 16 * 16 * 32

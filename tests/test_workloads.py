@@ -34,3 +34,12 @@ def test_per_query_selection_locality():
     near = sum(overlap(x[0, t], x[0, t + 1]) for t in range(0, 15))
     far = sum(overlap(x[0, t], x[0, t + 16]) for t in range(0, 15))
     assert near > 10 * 15 and far < 4 * 15
+
+
+def test_per_query_selection_large_locality():
+    x = W.per_query_selection_large(3, 2, 64, 5000, 64, group=16, shared=0.75)
+    assert x.shape == (2, 64, 64) and x.dtype == torch.int32
+    assert bool((x[..., 1:] >= x[..., :-1]).all()) and int(x.min()) >= 0 and int(x.max()) < 5000
+    near = len(set(x[0, 0].tolist()) & set(x[0, 1].tolist()))
+    far = len(set(x[0, 0].tolist()) & set(x[0, 40].tolist()))
+    assert near > 30 and far < 8
