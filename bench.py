@@ -51,9 +51,9 @@ def launches_per_step(w):
     att = 2 if small or w.dtype == "bf16" else 1
     return sel + att
 # DRAM traffic of one attention-kernel launch on the 128K-context workload
-# (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture, summarised in
-# profiles/attn_tc2_kernel_ctx_128k.md), valid only for the kernel sources it was taken
-# on: the digest below covers them, and a changed kernel reports null.
+# (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture of that kernel alone,
+# one launch, on this workload), valid only for the kernel sources it was taken on: the
+# digest below covers them, and a changed kernel reports null.
 ATTN_TRAFFIC = {"workload": "ctx_128k", "bytes": 117.494272e6 + 21.887744e6,
                 "sources": ['query_oriented_sparse_b200/csrc/attn_tc2.cuh', 'query_oriented_sparse_b200/csrc/tc_ptx.cuh'], "sha256_16": "e4300237fdf2f4d5"}
 
@@ -93,6 +93,57 @@ def stage_model(w: W.Workload):
                                 w.h_kv * n * 4)
         st["attn"]["flops"] += 4.0 * d * w.h_q * (C * n + C * (C + 1) / 2)
     return st
+
+
+KERNEL_STAGE = {"qsub_kernel": "qsub", "score_tc_kernel": "score", "score_simt_kernel": "score",
+                "score_decode_kernel": "score", "topk_kernel": "topk", "topk_block_kernel": "topk",
+                "attn_tc2_kernel": "attn", "attn_tc_kernel": "attn", "attn_simt_kernel": "attn",
+                "attn_decode_kernel": "attn"}
+
+
+def kernel_work(w, name):
+    """Algorithmic (flops, bytes) of one launch of a kernel of the chunk step.
+
+    The method's stages take their compulsory work (stage_model).  Two kernels move
+    bytes the method itself does not need, and are held to the bytes they must move:
+    top-k reads the pooled scores (4 B per key and column group) and writes idx, and
+    the compaction reads and writes every selected and chunk K/V row once."""
+    s, d, C = w.elem_bytes, w.head_dim, w.chunk
+    st = stage_model(w)
+    if name in ("topk_kernel", "topk_block_kernel"):
+        return 0.0, sum(w.h_kv * (P * 4 + min(B, P) * 4) for P, B in zip(w.prefix, w.budget))
+    if name == "compact_kv_kernel":
+        return 0.0, sum(2 * 2 * w.h_kv * (min(B, P) + C) * d * s
+                        for P, B in zip(w.prefix, w.budget))
+    stage = KERNEL_STAGE.get(name)
+    if stage is None:
+        return 0.0, 0.0
+    return st[stage]["flops"], st[stage]["bytes"]
+
+
+def kernel_table(w, times, peaks):
+    """Mean device time of each kernel over the profiled steps, with its roofline."""
+    acc = {}
+    for step in times:
+        for name, ms in step:
+            acc.setdefault(name, []).append(ms)
+    out = {}
+    for name, ms in acc.items():
+        n_per_step = len(ms) / len(times)
+        t = sum(ms) / len(times) / 1e3 / n_per_step        # per launch
+        fl, by = kernel_work(w, name)
+        t_fl = fl / (peaks["bf16_tflops"] * 1e12)
+        t_by = by / (peaks["hbm_gbs"] * 1e9)
+        row = {"us": t * 1e6, "launches_per_step": n_per_step}
+        if fl or by:
+            if t_fl >= t_by:
+                row.update(bound="tensor", achieved=fl / t / 1e12, unit="TFLOP/s",
+                           roofline_us=t_fl * 1e6, frac=t_fl / t)
+            else:
+                row.update(bound="hbm", achieved=by / t / 1e9, unit="GB/s",
+                           roofline_us=t_by * 1e6, frac=t_by / t)
+        out[name] = row
+    return out
 
 
 def attn_kernel_name(w):
@@ -364,6 +415,7 @@ def run_ours(args, w):
         select()
         attend()
     torch.cuda.synchronize()
+    select_eager, attend_eager = select, attend
     # Each call is captured once into a CUDA graph and replayed every step, as a serving
     # loop runs a fixed-shape step: the kernels are the same, the host's per-call work
     # (argument checks, tensor maps, ctypes marshalling) leaves the step.
@@ -405,6 +457,18 @@ def run_ours(args, w):
     step_ms = [a + b for a, b in zip(sel_ms, att_ms)]
     total_s = sum(step_ms) / 1e3
     assert Bd.device_error() == 0
+
+    # per-kernel device times: the same two calls launched eagerly, an event recorded
+    # after every kernel (outside the timed region above; same L2 flush before each step)
+    ktimes = []
+    for i in range(args.steps):
+        flush.zero_()
+        with Bd.KernelTimer(stream=stream) as kt:
+            select_eager()
+            attend_eager()
+        ktimes.append(kt.times)
+    assert Bd.device_error() == 0
+    kernels = kernel_table(w, ktimes, peaks)
 
     # end to end through host buffers and the serving call (quoka_step): every step's new
     # inputs (Q and the chunk's own K/V rows, packed [batch, h_kv, C, d]) go host->device
@@ -510,6 +574,8 @@ def run_ours(args, w):
         "gpu_launches": launches_per_step(w) * args.steps,
         "stage_us": {"select": statistics.mean(sel_ms) * 1e3,
                      "attn": statistics.mean(att_ms) * 1e3},
+        "kernel_us": {k: v["us"] for k, v in kernels.items()},
+        "kernels": kernels,
         "roofline": roof,
         "path_roofline": {"roofline_us": path_roof_us, "stage_roofline_us": rl,
                           "measured_us": total_s * 1e6 / args.steps,
@@ -800,7 +866,9 @@ def run_perq(args):
     w = W.WORKLOADS["ctx_128k"]
     t = W.generate(w)
     n_rows = t.kv_off[1]
-    sel_h = W.per_query_selection_large(7, w.h_q, w.chunk, n_rows, PERQ_S, group=PERQ_GROUP)
+    # causal sets: query t draws from the prefix and the chunk rows up to its own
+    sel_h = W.per_query_selection_large(7, w.h_q, w.chunk, n_rows, PERQ_S, group=PERQ_GROUP,
+                                        causal_prefix=w.prefix[0])
     tq = max(1, 16 // w.group)
     union_rows, flat_rows = perq_union_rows(sel_h, w.h_kv, tq)
     q, k, v = t.q.to(dev), t.k_cache.to(dev), t.v_cache.to(dev)
@@ -847,6 +915,7 @@ def run_perq(args):
         "data": "synthetic",
         "config": {"workload": "perq_128k", "chunk": w.chunk, "cache_rows": n_rows,
                    "h_q": w.h_q, "h_kv": w.h_kv, "head_dim": w.head_dim, "keys_per_query": PERQ_S,
+                   "causal": True,
                    "locality_group": PERQ_GROUP, "tile_rows": w.group * tq,
                    "l2": "256 MB flush before every timed call",
                    "launch": "CUDA graph, captured once and replayed every step"},

@@ -286,8 +286,9 @@ size_t quoka_prefill_workspace_size(const quoka_shape* shape, int n_chunks, int 
  * the library, reserved on every GPU that loads the library until the process
  * exits.  A call whose quoka_select_workspace_size() would exceed that size returns
  * QUOKA_ERR_WORKSPACE and launches nothing.  The first call on a device looks up the
- * array's device address (once per device, with that device current); make that
- * first call before any stream capture.  All calls share the one array and the
+ * array's device address (once per device and context, with that device current);
+ * make that first call before any stream capture.  After cudaDeviceReset the next
+ * call sees a new context and looks the address up again.  All calls share the one array and the
  * kernels overwrite every scratch byte they read, so nothing needs clearing between
  * calls - but two calls whose kernels overlap on the GPU (different streams without
  * ordering between them) race on the array.  The library allocates nothing here.
@@ -297,6 +298,30 @@ quoka_status quoka_select_noalloc(const quoka_shape* shape, const void* q_chunk,
                                   const void* k_cache, const int64_t* kv_off,
                                   const int32_t* prefix_len, int nq, const int32_t* budget,
                                   int b_max, int32_t* idx_out, int32_t* kept_out, void* stream);
+
+/*
+ * quoka_profile_events - per-kernel timing, for diagnostics and benchmarks.
+ *
+ * The paper has no counterpart to this call.  `events` is an array of `n_events`
+ * caller-created CUDA events (cudaEvent_t handles created with timing enabled and
+ * already valid on the device of the calls), or NULL to stop.  While an array is set
+ * on the calling thread, every kernel the library launches from that thread is
+ * followed by a cudaEventRecord of the next unused event on the launch's stream, until
+ * all n_events are used; a caller that records its own event on the stream before a
+ * call gets each kernel's time as the gap between consecutive events.  The caller owns
+ * the events (the library only records them) and must keep the array alive while it
+ * is set.  Do not set an array while capturing a stream into a graph.  Setting an
+ * array, or NULL, resets the count.  Returns QUOKA_ERR_INVALID_ARG for n_events < 1
+ * or a NULL handle.
+ */
+quoka_status quoka_profile_events(void* const* events, int n_events);
+
+/*
+ * How many events the launches recorded since quoka_profile_events on this thread;
+ * names[i] (for i < max_names; names may be NULL) receives the name of the kernel whose
+ * launch recorded event i (static strings owned by the library).
+ */
+int quoka_profile_marks(const char** names, int max_names);
 
 /* Thread-local description of the last non-OK status returned on this thread. */
 const char* quoka_last_error(void);

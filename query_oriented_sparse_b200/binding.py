@@ -60,6 +60,8 @@ SIGNATURES = {
                                      ctypes.c_size_t, _P]),
     "quoka_prefill_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int, ctypes.c_int,
                                                        ctypes.c_int]),
+    "quoka_profile_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
+    "quoka_profile_marks": (ctypes.c_int, [ctypes.POINTER(ctypes.c_char_p), ctypes.c_int]),
 }
 
 _lib = None
@@ -299,3 +301,41 @@ def device_error(stream: Optional[torch.cuda.Stream] = None) -> int:
     code = ctypes.c_uint32(0)
     _check(lib().quoka_device_error(ctypes.byref(code), ctypes.c_void_p(_stream(stream))))
     return code.value
+
+
+class KernelTimer:
+    """Per-kernel device times of the library calls made inside a ``with`` block.
+
+    Records a start event on the stream, hands the library a pool of timing events (one
+    is recorded after every kernel it launches from this thread, quoka_profile_events),
+    and afterwards yields (kernel name, milliseconds) pairs in launch order.  Eager calls
+    only: not inside a stream capture.
+    """
+
+    def __init__(self, max_kernels: int = 64, stream: Optional[torch.cuda.Stream] = None):
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        self.start = torch.cuda.Event(enable_timing=True)
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(max_kernels)]
+        for e in [self.start] + self.events:          # torch creates events on first record
+            e.record(self.stream)
+        self.stream.synchronize()
+        self._handles = (ctypes.c_void_p * max_kernels)(*[e.cuda_event for e in self.events])
+        self.times = []
+
+    def __enter__(self):
+        self.start.record(self.stream)
+        _check(lib().quoka_profile_events(self._handles, len(self.events)))
+        return self
+
+    def __exit__(self, *exc):
+        n = int(lib().quoka_profile_marks(None, 0))
+        names = (ctypes.c_char_p * max(n, 1))()
+        lib().quoka_profile_marks(names, n)
+        _check(lib().quoka_profile_events(None, 0))
+        if exc[0] is None:
+            self.stream.synchronize()
+            prev = self.start
+            for i in range(n):
+                self.times.append((names[i].decode(), prev.elapsed_time(self.events[i])))
+                prev = self.events[i]
+        return False

@@ -43,6 +43,23 @@ quoka_status cuda_fail(cudaError_t e, const char* where) {
   return fail(QUOKA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
 
+// Per-kernel timing (quoka_profile_events): while a caller's event array is set on this
+// thread, every launch is followed by a record of the next event on the launch's stream.
+struct ProfState {
+  void* const* events = nullptr;
+  int n = 0, used = 0;
+  std::vector<const char*> names;
+};
+thread_local ProfState g_prof;
+
+void prof_mark(cudaStream_t st, const char* name) {
+  if (!g_prof.events || g_prof.used >= g_prof.n) return;
+  if (cudaEventRecord(reinterpret_cast<cudaEvent_t>(g_prof.events[g_prof.used]), st) != cudaSuccess)
+    return;
+  g_prof.names.push_back(name);
+  ++g_prof.used;
+}
+
 struct Dims {
   int batch, h_q, h_kv, G, D, C;
   quoka_dtype dt;
@@ -261,6 +278,7 @@ quoka_status launch_score_tc(const Dims& d, const SeqTable& tab, long long rows,
       kmap, qmap, tab, p, reinterpret_cast<const float*>(ws + w.qinv),
       reinterpret_cast<const float*>(ws + w.qbias), reinterpret_cast<float*>(ws + w.pooled));
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score_tc launch");
+  prof_mark(st, "score_tc_kernel");
   return QUOKA_OK;
 }
 
@@ -276,6 +294,7 @@ quoka_status launch_topk(const Dims& d, const SeqTable& tab, int b_max, int32_t*
     topk_block_kernel<<<nrows, 512, smem, st>>>(pooled, w.pooled_stride, w.ncg, w.cg_stride,
                                                  1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk_block launch");
+    prof_mark(st, "topk_block_kernel");
     return QUOKA_OK;
   }
   const int tk_keys = std::min((tab.max_prefix + TOPK_CS - 1) / TOPK_CS, TOPK_STAGE_KEYS);
@@ -285,6 +304,7 @@ quoka_status launch_topk(const Dims& d, const SeqTable& tab, int b_max, int32_t*
   topk_kernel<<<nrows * TOPK_CS, TOPK_THREADS, tk_smem, st>>>(
       pooled, w.pooled_stride, w.ncg, w.cg_stride, 1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
+  prof_mark(st, "topk_kernel");
   return QUOKA_OK;
 }
 
@@ -300,6 +320,7 @@ quoka_status launch_score_decode_r(const Dims& d, const SeqTable& tab, long long
       reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(k), rows, tab, d.h_q, d.h_kv, d.C,
       pooled, w.pooled_stride);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score_decode launch");
+  prof_mark(st, "score_decode_kernel");
   return QUOKA_OK;
 }
 
@@ -315,6 +336,7 @@ quoka_status launch_select_decode(const Dims& d, const SeqTable& tab, long long 
     const int grid = (int)std::min<long long>((n + 255) / 256, (long long)sm_count() * 4);
     kept_all_kernel<<<grid, 256, 0, st>>>(kept_out, d.batch * d.h_q, d.C, nq);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "kept launch");
+    prof_mark(st, "kept_all_kernel");
   }
   if (tab.max_prefix == 0) return QUOKA_OK;
   int r = 1;
@@ -349,6 +371,7 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
   qsub_kernel<T, D><<<d.batch * d.h_q * QSUB_CS, QSUB_THREADS, qs_smem, st>>>(
       reinterpret_cast<const T*>(q), d.C, w.nk, w.nkp, nq, kept_out, qsel, qinv, qbias);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "qsub launch");
+  prof_mark(st, "qsub_kernel");
 
   if (tab.max_prefix > 0) {
     if (w.tc) {
@@ -362,6 +385,7 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
           reinterpret_cast<const T*>(k), rows, tab, d.h_kv, d.G, w.nkp, qsel, qinv, qbias, pooled,
           w.pooled_stride);
       if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score launch");
+      prof_mark(st, "score_simt_kernel");
     }
   }
 
@@ -424,6 +448,7 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
       reinterpret_cast<const uint4*>(k_new), reinterpret_cast<const uint4*>(v_new),
       reinterpret_cast<uint4*>(const_cast<void*>(k)), reinterpret_cast<uint4*>(const_cast<void*>(v)));
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "compact launch");
+  prof_mark(st, "compact_kv_kernel");
   // 2. dense attention over it
   CUtensorMap qmap, kmap, vmap;
   quoka_status s;
@@ -446,6 +471,7 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
     attn_tc2_kernel<<<grid2, AT2_THREADS, smem2, st>>>(qmap, kmap, vmap, tab, p2,
                                                        reinterpret_cast<__nv_bfloat16*>(out));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_tc2 launch");
+    prof_mark(st, "attn_tc2_kernel");
     return QUOKA_OK;
   }
   if ((s = make_map_bf16(&kmap, kc, kc_rows, D, 64, 128, "compacted K")) != QUOKA_OK) return s;
@@ -456,6 +482,7 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
   attn_tc_kernel<D><<<grid, ATC_THREADS, smem, st>>>(qmap, kmap, vmap, tab, p,
                                                       reinterpret_cast<__nv_bfloat16*>(out));
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_tc launch");
+  prof_mark(st, "attn_tc_kernel");
   return QUOKA_OK;
 }
 
@@ -486,9 +513,11 @@ quoka_status launch_attn_decode_r(const Dims& d, const SeqTable& tab, long long 
       reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(k), reinterpret_cast<const T*>(v),
       rows, tab, d.h_q, d.h_kv, d.C, idx, b_max, (int)split, nsplit_ws, scale_log2, part);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode launch");
+  prof_mark(st, "attn_decode_kernel");
   attn_decode_combine_kernel<T, D, R><<<dim3(d.h_kv, d.batch), 128, 0, st>>>(
       part, tab, d.h_q, d.h_kv, d.C, (int)split, nsplit_ws, reinterpret_cast<T*>(out));
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  prof_mark(st, "attn_decode_combine_kernel");
   return QUOKA_OK;
 }
 
@@ -525,6 +554,7 @@ quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, con
         reinterpret_cast<uint4*>(const_cast<void*>(k)), reinterpret_cast<uint4*>(const_cast<void*>(v)),
         rows, tab, d.h_kv, d.C, vpr, vecs);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "append launch");
+    prof_mark(st, "append_kv_kernel");
   }
   if (decode) return launch_attn_decode<T, D>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
   const int s = attn_simt_smem_bytes<D>();
@@ -535,6 +565,7 @@ quoka_status launch_attn(const Dims& d, const SeqTable& tab, long long rows, con
       reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(k), reinterpret_cast<const T*>(v),
       rows, tab, d.h_q, d.h_kv, d.C, idx, b_max, reinterpret_cast<T*>(out), scale_log2);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn launch");
+  prof_mark(st, "attn_simt_kernel");
   return QUOKA_OK;
 }
 
@@ -586,6 +617,7 @@ quoka_status launch_perq_r(const Dims& d, const SeqTable& tab, long long rows, c
   perq_union_kernel<<<dim3(pl.ntiles, d.h_kv, d.batch), PQ_UNION_THREADS, usmem, st>>>(
       sel, tab, d.h_q, d.h_kv, d.C, S, pl.TQ, uni, memb, ucount);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_union launch");
+  prof_mark(st, "perq_union_kernel");
   const int smem = adc_smem_bytes<T, D, R>();
   if ((e = ensure_smem(perq_attn_kernel<T, D, R>, smem)) != cudaSuccess) return cuda_fail(e, "perq_attn smem");
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
@@ -594,9 +626,11 @@ quoka_status launch_perq_r(const Dims& d, const SeqTable& tab, long long rows, c
       rows, tab, d.h_q, d.h_kv, d.C, S, pl.TQ, uni, memb, ucount, pl.split, pl.nsplit, scale_log2,
       part);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_attn launch");
+  prof_mark(st, "perq_attn_kernel");
   perq_combine_kernel<T, D, R><<<dim3(pl.ntiles, d.batch * d.h_kv), 128, 0, st>>>(
       part, ucount, d.h_q, d.h_kv, d.C, pl.TQ, pl.split, pl.nsplit, reinterpret_cast<T*>(out));
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_combine launch");
+  prof_mark(st, "perq_combine_kernel");
   return QUOKA_OK;
 }
 
@@ -661,7 +695,25 @@ quoka_status run_prefill(const Dims& d, int n_chunks, const unsigned char* q, co
 
 extern "C" {
 
-int quoka_version(void) { return 100; }
+int quoka_version(void) { return 101; }
+
+quoka_status quoka_profile_events(void* const* events, int n_events) {
+  if (events && n_events < 1) return fail(QUOKA_ERR_INVALID_ARG, "n_events must be >= 1");
+  if (events)
+    for (int i = 0; i < n_events; ++i)
+      if (!events[i]) return fail(QUOKA_ERR_INVALID_ARG, "events[%d] is NULL", i);
+  g_prof.events = events;
+  g_prof.n = events ? n_events : 0;
+  g_prof.used = 0;
+  g_prof.names.clear();
+  return QUOKA_OK;
+}
+
+int quoka_profile_marks(const char** names, int max_names) {
+  const int n = g_prof.used;
+  for (int i = 0; names && i < n && i < max_names; ++i) names[i] = g_prof.names[i];
+  return n;
+}
 
 const char* quoka_last_error(void) { return g_last_error.c_str(); }
 
@@ -910,21 +962,55 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[QUOKA_NOALLOC_S
 
 namespace {
 std::mutex g_noalloc_mu;
-std::map<int, void*> g_noalloc_addr;  // device ordinal -> device address of the array
+// (device ordinal, unique ID of the context current on it) -> device address of the
+// array.  A device reset destroys the primary context and the next one loads the module
+// again, possibly elsewhere; its new context ID makes the lookup run again.
+std::map<std::pair<int, unsigned long long>, void*> g_noalloc_addr;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique ID of the calling thread's current context (0 if the driver cannot say).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur && get_id && get_cur(&ctx) == CUDA_SUCCESS && ctx) get_id(ctx, &id);
+  return id;
+}
 
 quoka_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  auto it = g_noalloc_addr.find(dev);
-  if (it == g_noalloc_addr.end()) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
-    it = g_noalloc_addr.emplace(dev, p).first;
+  unsigned long long id = current_context_id();
+  if (id != 0) {
+    auto it = g_noalloc_addr.find(std::make_pair(dev, id));
+    if (it != g_noalloc_addr.end()) {
+      *out = it->second;
+      return QUOKA_OK;
+    }
   }
-  *out = it->second;
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // creates the context if need be
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
+  id = current_context_id();
+  if (id != 0) g_noalloc_addr[std::make_pair(dev, id)] = p;   // else: looked up every call
+  *out = p;
   return QUOKA_OK;
 }
 }  // namespace

@@ -243,19 +243,31 @@ def per_query_selection(seed: int, h_q: int, n_queries: int, n_keys: int, s: int
 
 
 def per_query_selection_large(seed: int, h_q: int, n_queries: int, n_keys: int, s: int,
-                              group: int = 16, shared: float = 0.75) -> torch.Tensor:
+                              group: int = 16, shared: float = 0.75,
+                              causal_prefix=None) -> torch.Tensor:
     """per_query_selection for large sizes, vectorised per head: every run of `group`
     consecutive queries draws one base set; each entry of a query's set is the base
     set's entry at that slot with probability `shared`, else a draw of its own.  Draws
     are with replacement, so a set may hold a position twice (the attention counts it
-    once).  Returns int32 [h_q, n_queries, s], rows ascending."""
+    once).  With `causal_prefix` = P, query t draws only from rows 0 .. P + t (the
+    prefix and the chunk rows up to its own), the base set of a run from the rows its
+    first query may see; else from all n_keys rows.  Returns int32 [h_q, n_queries, s],
+    rows ascending."""
     g = torch.Generator(device="cpu").manual_seed(seed)
     ngroups = (n_queries + group - 1) // group
     gid = torch.arange(n_queries) // group
+    if causal_prefix is None:
+        lim_q = torch.full((n_queries, 1), n_keys, dtype=torch.float64)
+        lim_g = torch.full((ngroups, 1), n_keys, dtype=torch.float64)
+    else:
+        lim_q = (causal_prefix + 1 + torch.arange(n_queries, dtype=torch.float64))[:, None]
+        lim_g = (causal_prefix + 1 + group * torch.arange(ngroups, dtype=torch.float64))[:, None]
+        if causal_prefix + n_queries > n_keys:
+            raise ValueError("causal_prefix + n_queries exceeds n_keys")
     out = torch.empty(h_q, n_queries, s, dtype=torch.int32)
     for h in range(h_q):
-        base = torch.randint(0, n_keys, (ngroups, s), generator=g)
-        own = torch.randint(0, n_keys, (n_queries, s), generator=g)
+        base = (torch.rand(ngroups, s, generator=g, dtype=torch.float64) * lim_g).long()
+        own = (torch.rand(n_queries, s, generator=g, dtype=torch.float64) * lim_q).long()
         take = torch.rand(n_queries, s, generator=g) < shared
         rows = torch.where(take, base[gid], own)
         out[h] = torch.sort(rows, dim=1).values.to(torch.int32)

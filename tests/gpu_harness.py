@@ -9,7 +9,7 @@ from query_oriented_sparse_b200 import binding as Bd
 from query_oriented_sparse_b200 import workloads as W
 
 from parity_util import (ATTN_TOL, check_index_row, compare_kept_set, compare_top_set,
-                         row_rel_err)
+                         row_rel_err, stratified_rows)
 
 
 def run_gpu(w: W.Workload, t: W.Tensors, chunk_index: int = 0, device="cuda"):
@@ -44,8 +44,9 @@ def run_gpu(w: W.Workload, t: W.Tensors, chunk_index: int = 0, device="cuda"):
 def check_step(w: W.Workload, t: W.Tensors, res, chunk_index: int = 0, attn_rows=None):
     """Asserts parity of one chunk step; returns a report dict.
 
-    attn_rows: None for every output row, else an int giving the number of sampled
-    (head, position) rows per sequence (plus the first and last position of head 0).
+    attn_rows: None for every output row, or "tiles" for one row of every query tile of
+    every KV head of every sequence plus each head's first and last position of the
+    last tile (parity_util.stratified_rows).
     """
     assert res["device_error"] == 0
     report = {"kept_near_ties": 0, "idx_near_ties": 0, "max_pooled_err": 0.0,
@@ -89,9 +90,8 @@ def check_step(w: W.Workload, t: W.Tensors, res, chunk_index: int = 0, attn_rows
             o_ref = O.attend_chunk(q64, kseq, vseq, P, gpu_idx)
             e = row_rel_err(res["out"][b], o_ref)
         else:
-            rows = [(0, 0), (0, w.chunk - 1), (w.h_q - 1, w.chunk - 1)]
-            rows += [(int(rng.integers(w.h_q)), int(rng.integers(w.chunk)))
-                     for _ in range(attn_rows)]
+            assert attn_rows == "tiles", attn_rows
+            rows = stratified_rows(w.h_q, w.h_kv, w.chunk, rng)
             o_ref = O.attend_chunk(q64, kseq, vseq, P, gpu_idx, rows=rows)
             o_gpu = np.stack([res["out"][b, h, tt] for h, tt in rows])
             e = row_rel_err(o_gpu, o_ref)

@@ -65,6 +65,28 @@ def compare_kept_set(gpu: np.ndarray, cos: np.ndarray, nq: int) -> int:
     return int(diff.size)
 
 
+def stratified_rows(h_q: int, h_kv: int, C: int, rng) -> list:
+    """(head, position) rows that touch every query tile of the tensor-core attention.
+
+    A tile packs the G = h_q / h_kv query heads of one KV head at TP = 128 // G
+    consecutive positions (one CTA of an SM pair holds one tile).  Per KV head and per
+    tile this takes one row at a random head of the group and a random position of the
+    tile, and adds, for every head of the group, the first and the last position of the
+    last tile (its ragged tail, when C is not a multiple of TP).
+    """
+    G = h_q // h_kv
+    tp = max(1, 128 // G)
+    rows = []
+    for g in range(h_kv):
+        heads = range(g * G, (g + 1) * G)
+        for t0 in range(0, C, tp):
+            rows.append((g * G + int(rng.integers(G)), t0 + int(rng.integers(min(tp, C - t0)))))
+        last = (C - 1) // tp * tp
+        for h in heads:
+            rows += [(h, last), (h, C - 1)]
+    return sorted(set(rows))
+
+
 def row_rel_err(o: np.ndarray, ref: np.ndarray) -> float:
     """max over rows of |o - ref|_inf / |ref|_inf (rows along the last axis)."""
     o = np.asarray(o, dtype=np.float64).reshape(-1, o.shape[-1])

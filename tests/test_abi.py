@@ -36,7 +36,7 @@ def test_library_loads_and_exports_every_declared_symbol():
     for name in declared_functions():
         assert hasattr(lib, name), f"libquoka.so does not export {name}"
     assert set(declared_functions()) == set(Bd.SIGNATURES), "binding and header disagree"
-    assert Bd.version() == 100
+    assert Bd.version() == 101
 
 
 def test_attn_workspace_size():
@@ -220,3 +220,14 @@ def test_noalloc_rejects_oversize_before_launch():
                                   None, None)
     assert st == Bd.QUOKA_ERR_WORKSPACE
     assert "built-in scratch" in lib.quoka_last_error().decode()
+
+
+def test_profile_events_host_checks():
+    """The timing hook checks its arguments on the host and starts with no marks."""
+    lib = Bd.lib()
+    assert lib.quoka_profile_events(None, 0) == Bd.QUOKA_OK
+    assert lib.quoka_profile_marks(None, 0) == 0
+    empty = (ctypes.c_void_p * 1)(None)
+    assert lib.quoka_profile_events(empty, 1) == Bd.QUOKA_ERR_INVALID_ARG
+    assert lib.quoka_profile_events(empty, 0) == Bd.QUOKA_ERR_INVALID_ARG
+    assert lib.quoka_profile_marks(None, 0) == 0

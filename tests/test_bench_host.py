@@ -106,3 +106,27 @@ def test_perq_union_rows_counts_distinct_per_tile():
     ref = sum(len(set(sel[4 * g:4 * g + 4, t0:t0 + 4].flatten().tolist()))
               for g in range(2) for t0 in range(0, 64, 4))
     assert u == ref and flat == 2 * 16 * 16 * 32
+
+
+def test_kernel_table_per_launch_rooflines():
+    """Per-kernel rows: mean time per launch, the stage's algorithmic work, its bound."""
+    w = W.WORKLOADS["ctx_128k"]
+    peaks = {"hbm_gbs": 6440.7, "bf16_tflops": 1687.0, "bf16_tflops_sustained": 1436.0}
+    steps = [[("qsub_kernel", 0.026), ("score_tc_kernel", 0.150), ("topk_kernel", 0.020),
+              ("compact_kv_kernel", 0.024), ("attn_tc2_kernel", 1.090)]] * 3
+    tab = bench.kernel_table(w, steps, peaks)
+    assert list(tab) == ["qsub_kernel", "score_tc_kernel", "topk_kernel", "compact_kv_kernel",
+                         "attn_tc2_kernel"]
+    a = tab["attn_tc2_kernel"]
+    assert a["bound"] == "tensor" and abs(a["us"] - 1090.0) < 1e-6
+    assert abs(a["roofline_us"] - 733.24) < 0.1 and abs(a["frac"] - 733.24 / 1090.0) < 1e-3
+    sc = tab["score_tc_kernel"]
+    assert sc["bound"] == "tensor" and abs(sc["roofline_us"] - 81.47) < 0.1
+    tk = tab["topk_kernel"]
+    assert tk["bound"] == "hbm"
+    assert abs(tk["achieved"] - (8 * (131072 + 16384) * 4) / 20e-6 / 1e9) < 1e-6
+    cp = tab["compact_kv_kernel"]
+    assert abs(cp["achieved"] - 2 * 2 * 8 * (16384 + 4096) * 256 / 24e-6 / 1e9) < 1e-6
+    # a kernel launched twice per step is reported per launch
+    tab2 = bench.kernel_table(w, [[("qsub_kernel", 0.01), ("qsub_kernel", 0.03)]], peaks)
+    assert abs(tab2["qsub_kernel"]["us"] - 20.0) < 1e-9 and tab2["qsub_kernel"]["launches_per_step"] == 2

@@ -393,12 +393,62 @@ def pin_prefill_is_causal_over_chunks(seed=13):
             assert a.tolist() == b.tolist()
 
 
+def pin_batch_is_per_sequence(seed=16):
+    """A ragged batch in one shared cache: sequence b owns rows kv_off[b] .. kv_off[b+1]-1
+    (its prefix, its chunk rows at kv_off[b] + P_b + t, then rows nobody reads), and rows
+    before kv_off[0] belong to no sequence.  select_batch / attend_batch must give, per
+    sequence, what select_chunk / attend_chunk give on that sequence's own arrays, built
+    apart before the cache is assembled; rewriting the unread rows or another sequence's
+    rows changes nothing."""
+    rng = np.random.default_rng(seed)
+    H_q, H_kv, C, d, nq = 4, 2, 3, 6, 2
+    prefix = [7, 0, 11]
+    budget = [3, 2, 11]
+    junk = [2, 4, 1]
+    lead = 5
+    q = rng.normal(size=(len(prefix), H_q, C, d))
+    seq_k = [rng.normal(size=(H_kv, P + C, d)) for P in prefix]
+    seq_v = [rng.normal(size=(H_kv, P + C, d)) for P in prefix]
+
+    def assemble(fill):
+        ks, vs, off = [fill((H_kv, lead, d))], [fill((H_kv, lead, d))], [lead]
+        for b, P in enumerate(prefix):
+            ks += [seq_k[b], fill((H_kv, junk[b], d))]
+            vs += [seq_v[b], fill((H_kv, junk[b], d))]
+            off.append(off[-1] + P + C + junk[b])
+        return np.concatenate(ks, axis=1), np.concatenate(vs, axis=1), off
+
+    k, v, kv_off = assemble(lambda shp: rng.normal(size=shp))
+    sel = O.select_batch(q, k, kv_off, prefix, nq, budget)
+    out = O.attend_batch(q, k, v, kv_off, prefix, [r["idx"] for r in sel])
+    for b, P in enumerate(prefix):
+        ref = O.select_chunk(q[b], seq_k[b], P, nq, budget[b])
+        for g in range(H_kv):
+            assert sel[b]["idx"][g].tolist() == ref["idx"][g].tolist(), (b, g)
+            assert sel[b]["idx"][g].size == min(budget[b], P)
+        np.testing.assert_array_equal(sel[b]["score"], ref["score"])
+        np.testing.assert_array_equal(out[b], O.attend_chunk(q[b], seq_k[b], seq_v[b], P, ref["idx"]))
+    # unread rows rewritten: nothing moves
+    k2, v2, _ = assemble(lambda shp: 100.0 * rng.normal(size=shp))
+    sel2 = O.select_batch(q, k2, kv_off, prefix, nq, budget)
+    np.testing.assert_array_equal(O.attend_batch(q, k2, v2, kv_off, prefix,
+                                                 [r["idx"] for r in sel2]), out)
+    # another sequence's rows rewritten: sequences 0 and 1 keep their results
+    k3, v3 = k.copy(), v.copy()
+    k3[:, kv_off[2]:kv_off[3]] = rng.normal(size=k3[:, kv_off[2]:kv_off[3]].shape)
+    v3[:, kv_off[2]:kv_off[3]] = rng.normal(size=v3[:, kv_off[2]:kv_off[3]].shape)
+    sel3 = O.select_batch(q, k3, kv_off, prefix, nq, budget)
+    out3 = O.attend_batch(q, k3, v3, kv_off, prefix, [r["idx"] for r in sel3])
+    np.testing.assert_array_equal(out3[:2], out[:2])
+    assert not np.array_equal(out3[2], out[2])
+
+
 ALL_PINS = [pin_query_cosine_closed_form, pin_subselect_brute_force, pin_query_scale_invariance,
             pin_scoring_closed_forms, pin_key_scale_and_permutation, pin_top_budget_brute_force,
             pin_worked_example, pin_attention_vs_sdpa, pin_full_budget_is_full_causal,
             pin_gqa_is_independent_mqa, pin_prefill_full_budget_is_causal,
             pin_prefill_zero_budget_is_block_causal, pin_prefill_is_causal_over_chunks,
-            pin_decode_is_mean_cosine, pin_per_query_vs_sdpa]
+            pin_decode_is_mean_cosine, pin_per_query_vs_sdpa, pin_batch_is_per_sequence]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
@@ -606,11 +656,24 @@ def _mut_per_query_reads_padding(mp):
     mp.setattr(O, "attend_per_query", _per_query_variant(dedupe=True, drop_padding=False))
 
 
+def _mut_seq_rows_off_by_one(mp):
+    """A sequence's rows taken one row late."""
+    mp.setattr(O, "_seq_rows", lambda x, kv_off, b: x[:, kv_off[b] + 1:kv_off[b + 1] + 1])
+
+
+def _mut_batch_budget_of_next_sequence(mp):
+    """Each sequence selected with the next sequence's budget."""
+    orig = O.select_batch
+    mp.setattr(O, "select_batch", lambda q, k, kv_off, prefix, nq, budget:
+               orig(q, k, kv_off, prefix, nq, list(budget[1:]) + list(budget[:1])))
+
+
 MUTANTS = [_mut_most_similar, _mut_raw_mean, _mut_max_over_group, _mut_mean_then_max,
            _mut_no_key_norm, _mut_ties_high_index, _mut_no_softmax_scale,
            _mut_causal_excludes_self, _mut_prefill_own_chunk_candidates,
            _mut_prefill_budget_shift, _mut_per_query_counts_duplicates,
-           _mut_per_query_reads_padding]
+           _mut_per_query_reads_padding, _mut_seq_rows_off_by_one,
+           _mut_batch_budget_of_next_sequence]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)

@@ -1,8 +1,8 @@
 """Per-query sparse attention with shared loading (QUILT page, summary): every query
 attends to its own key set, tiles of up to 16 rows load the union of their sets once.
 Checked row by row against the oracle's per-query attention, across both dtypes and head
-sizes, group sizes 1 to 16, ragged tiles, ragged batches, padding, duplicate entries and
-an empty set (zeros)."""
+sizes, group sizes 1 to 16 (3 and 12 leave padding rows in every tile), ragged tiles,
+ragged batches, padding, duplicate entries and an empty set (zeros)."""
 import numpy as np
 import pytest
 import torch
@@ -26,6 +26,11 @@ CASES = [
         seed=63), 200),
     (C_("pq_bf16_d128_g1_long", h_q=2, h_kv=2, head_dim=128, chunk=50, prefix=40000, nq=1,
         budget=1, recipe="heavy", seed=64), 64),
+    # group sizes that do not divide the 16-row tile: rows G * TQ .. 15 are padding
+    (C_("pq_bf16_d128_g3_ragged", h_q=6, h_kv=2, head_dim=128, chunk=23, prefix=(700, 90),
+        nq=1, budget=1, recipe="rank4", seed=65), 24),
+    (C_("pq_f32_d128_g12", h_q=12, h_kv=1, head_dim=128, chunk=9, prefix=1500, nq=1, budget=1,
+        dtype="f32", seed=66), 40),
 ]
 
 

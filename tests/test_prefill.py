@@ -17,7 +17,8 @@ from oracle import quoka_oracle as O
 from query_oriented_sparse_b200 import binding as Bd
 from query_oriented_sparse_b200 import workloads as W
 
-from parity_util import ATTN_TOL, check_index_row, compare_kept_set, compare_top_set, row_rel_err
+from parity_util import (ATTN_TOL, check_index_row, compare_kept_set, compare_top_set,
+                         row_rel_err, stratified_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -112,8 +113,9 @@ def run_by_hand(w, budgets, q, kn, vn, k0, v0, kv_off, dev):
 def check_chunk(w, c, budget, q, kn, vn, out_c, idx_c, kept_c, attn_rows=None):
     """Oracle parity of chunk c of the prompt: the GPU's kept queries and selected keys
     against the oracle's (near-ties counted and returned), then its output against the
-    oracle's attention over the GPU's selection (every row, or `attn_rows` sampled rows
-    plus the first and last)."""
+    oracle's attention over the GPU's selection (every row, or with attn_rows="tiles"
+    one row of every query tile of every KV head plus the last tile's first and last
+    position of every head)."""
     C = w.chunk
     P = c * C
     nk = min(w.nq, C)
@@ -141,8 +143,8 @@ def check_chunk(w, c, budget, q, kn, vn, out_c, idx_c, kept_c, attn_rows=None):
             o_ref = O.attend_chunk(qc, kp, vp, P, gpu_idx)
             e = row_rel_err(out_c[b].float().numpy(), o_ref)
         else:
-            rows = [(0, 0), (0, C - 1), (w.h_q - 1, C - 1)]
-            rows += [(int(rng.integers(w.h_q)), int(rng.integers(C))) for _ in range(attn_rows)]
+            assert attn_rows == "tiles", attn_rows
+            rows = stratified_rows(w.h_q, w.h_kv, C, rng)
             o_ref = O.attend_chunk(qc, kp, vp, P, gpu_idx, rows=rows)
             e = row_rel_err(np.stack([out_c[b, h, t].float().numpy() for h, t in rows]), o_ref)
         assert e <= tol, f"chunk {c} sequence {b}: rel err {e} > {tol}"
@@ -229,7 +231,8 @@ def test_prefill_rejections_launch_nothing(cuda_device):
 def test_prefill_full_size_prompt(cuda_device):
     """The 128K-context prompt (33 chunks of 4096) as the prefill benchmark runs it:
     every chunk bit-identical to the single-chunk calls, the cache filled with the
-    prompt, and oracle parity of the second and the last chunk (sampled attention rows)."""
+    prompt, and oracle parity of the second and the last chunk (one attention row of
+    every query tile)."""
     w = W.PROMPTS["prompt_128k"]
     budgets = w.budgets_of_chunks()
     t = W.generate(w)
@@ -270,5 +273,5 @@ def test_prefill_full_size_prompt(cuda_device):
     del qd, knd, vnd, k, v, k2, v2, out
     for c in kept_of:
         near = check_chunk(w, c, budgets[c], q, kn, vn, out_h[c], idx_of[c], kept_of[c],
-                           attn_rows=96)
+                           attn_rows="tiles")
         print("prompt_128k chunk", c, "near-ties", near)

@@ -43,3 +43,13 @@ def test_per_query_selection_large_locality():
     near = len(set(x[0, 0].tolist()) & set(x[0, 1].tolist()))
     far = len(set(x[0, 0].tolist()) & set(x[0, 40].tolist()))
     assert near > 30 and far < 8
+
+
+def test_per_query_selection_large_causal():
+    """With causal_prefix = P, query t only draws rows 0 .. P + t."""
+    P, T = 300, 40
+    x = W.per_query_selection_large(4, 3, T, P + T, 50, group=16, shared=0.75, causal_prefix=P)
+    assert bool((x[..., 1:] >= x[..., :-1]).all()) and int(x.min()) >= 0
+    lim = P + torch.arange(T, dtype=torch.int32)
+    assert bool((x.max(dim=-1).values <= lim[None]).all())
+    assert bool((x[:, T - 1] > P).any())          # late queries do reach chunk rows
