@@ -42,6 +42,12 @@ set, so the oracle follows the method's steps in the pages' order:
    attends to exactly its own set of key positions, softmax(q k^T / sqrt(d)) v over
    that set.  This is what shared-query execution must reproduce, whatever grouping
    and union loading it uses.
+9. selected-value cache (SQD page, the sparse-attention paragraph: the top-k choice
+   scans the whole cache, attention runs over the chosen values kept where it runs, and
+   only the values not kept yet, the misses, are sent): the slot map after moving the
+   kept rows to a new selection.  The page does not say where a fetched row goes; the
+   reading here is that a row kept before and chosen again stays in its slot and the
+   misses, in ascending row order, fill the freed slots in ascending order.
 
 Readings where the pages are silent (each is listed with its reason in the design
 notes of the repository): the budget B counts prefix keys only and the chunk's own
@@ -63,7 +69,7 @@ import numpy as np
 __all__ = [
     "unit_rows", "mean_query", "query_cosines", "subselect_queries", "pooled_key_scores",
     "top_budget", "select_chunk", "attend_chunk", "select_batch", "attend_batch",
-    "prefill_prompt", "attend_per_query",
+    "prefill_prompt", "attend_per_query", "selected_value_slots",
 ]
 
 
@@ -308,3 +314,33 @@ def attend_per_query(q, k, v, sel) -> np.ndarray:
             p = np.exp(logits - logits.max())
             out[h, t] = (p @ v[g, keys]) / p.sum()
     return out
+
+
+def selected_value_slots(slots_prev, idx_new, n: int):
+    """Step 9: the slot map of a selected-value cache after moving it to a new selection.
+
+    slots_prev: the row each slot held (-1 for none); idx_new: the n rows now selected
+    (distinct); n: the live slots.  A slot below n whose row is selected again keeps it
+    (if two slots held the same row, the lower one); every other slot below n is free;
+    the misses (selected rows no live slot kept) go, in ascending order, into the free
+    slots in ascending order; slots from n on are emptied.
+    Returns (new slot map as a list, the misses in ascending order).
+    """
+    prev = [int(x) for x in slots_prev]
+    wanted = set(int(x) for x in list(idx_new)[:n])
+    assert len(wanted) == n, "the selection must name n distinct rows"
+    new = [-1] * len(prev)
+    kept = set()
+    free = []
+    for s in range(n):
+        r = prev[s] if s < len(prev) else -1
+        if r in wanted and r not in kept:
+            new[s] = r
+            kept.add(r)
+        else:
+            free.append(s)
+    misses = sorted(wanted - kept)
+    assert len(misses) == len(free)
+    for s, r in zip(free, misses):
+        new[s] = r
+    return new, misses

@@ -443,12 +443,52 @@ def pin_batch_is_per_sequence(seed=16):
     assert not np.array_equal(out3[2], out[2])
 
 
+def pin_selected_value_slots(seed=17):
+    """The selected-value cache's slot map: a hand-worked case, then on random cases the
+    held set equals the selection, kept rows never move, the misses are exactly the
+    selected rows not kept before and fill the freed slots in order, and slots past the
+    live range are empty.  Attention over the rows in slot order equals attention over
+    the ascending selection (the set, not the order, decides it)."""
+    new, miss = O.selected_value_slots([5, 9, 2, -1], [2, 3, 9], 3)
+    assert new == [3, 9, 2, -1] and miss == [3]
+    new, miss = O.selected_value_slots([4, 4, 7, 1], [1, 4], 2)       # row 4 held twice
+    assert new == [4, 1, -1, -1] and miss == [1]
+    rng = np.random.default_rng(seed)
+    for _ in range(200):
+        P = int(rng.integers(1, 40))
+        bm = int(rng.integers(1, 12))
+        prev = [-1] * bm
+        n0 = int(rng.integers(0, min(bm, P) + 1))
+        prev[:n0] = rng.choice(P, size=n0, replace=False).tolist()
+        n = int(rng.integers(0, min(bm, P) + 1))
+        idx = np.sort(rng.choice(P, size=n, replace=False))
+        new, miss = O.selected_value_slots(prev, idx, n)
+        assert sorted(new[:n]) == sorted(idx.tolist()) and all(x == -1 for x in new[n:])
+        live_prev = set(prev[:min(n0, n)])
+        for s_ in range(n):
+            if prev[s_] in set(idx.tolist()) and prev.index(prev[s_]) == s_:
+                assert new[s_] == prev[s_]
+        assert miss == sorted(set(idx.tolist()) - live_prev)
+        freed = [s_ for s_ in range(n) if new[s_] != prev[s_]]
+        assert [new[s_] for s_ in freed] == miss
+    # attention is a function of the selected set: slot order changes nothing
+    H_q, H_kv, C, P, d = 4, 2, 3, 12, 8
+    q = rng.normal(size=(H_q, C, d))
+    k = rng.normal(size=(H_kv, P + C, d))
+    v = rng.normal(size=(H_kv, P + C, d))
+    sel = [np.sort(rng.choice(P, size=5, replace=False)) for _ in range(H_kv)]
+    shuffled = [rng.permutation(x) for x in sel]
+    np.testing.assert_allclose(O.attend_chunk(q, k, v, P, shuffled), O.attend_chunk(q, k, v, P, sel),
+                               rtol=1e-12, atol=1e-13)
+
+
 ALL_PINS = [pin_query_cosine_closed_form, pin_subselect_brute_force, pin_query_scale_invariance,
             pin_scoring_closed_forms, pin_key_scale_and_permutation, pin_top_budget_brute_force,
             pin_worked_example, pin_attention_vs_sdpa, pin_full_budget_is_full_causal,
             pin_gqa_is_independent_mqa, pin_prefill_full_budget_is_causal,
             pin_prefill_zero_budget_is_block_causal, pin_prefill_is_causal_over_chunks,
-            pin_decode_is_mean_cosine, pin_per_query_vs_sdpa, pin_batch_is_per_sequence]
+            pin_decode_is_mean_cosine, pin_per_query_vs_sdpa, pin_batch_is_per_sequence,
+            pin_selected_value_slots]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
@@ -668,12 +708,33 @@ def _mut_batch_budget_of_next_sequence(mp):
                orig(q, k, kv_off, prefix, nq, list(budget[1:]) + list(budget[:1])))
 
 
+def _mut_slots_misses_descending(mp):
+    """Misses placed into the freed slots in descending row order."""
+    orig = O.selected_value_slots
+    def bad(prev, idx, n):
+        new, miss = orig(prev, idx, n)
+        freed = [s for s in range(n) if new[s] in miss]
+        for s, r in zip(freed, sorted(miss, reverse=True)):
+            new[s] = r
+        return new, miss
+    mp.setattr(O, "selected_value_slots", bad)
+
+
+def _mut_slots_refetch_hits(mp):
+    """Every selected row fetched again into ascending slots (hits not kept)."""
+    def bad(prev, idx, n):
+        rows = sorted(int(x) for x in list(idx)[:n])
+        return rows + [-1] * (len(prev) - n), rows
+    mp.setattr(O, "selected_value_slots", bad)
+
+
 MUTANTS = [_mut_most_similar, _mut_raw_mean, _mut_max_over_group, _mut_mean_then_max,
            _mut_no_key_norm, _mut_ties_high_index, _mut_no_softmax_scale,
            _mut_causal_excludes_self, _mut_prefill_own_chunk_candidates,
            _mut_prefill_budget_shift, _mut_per_query_counts_duplicates,
            _mut_per_query_reads_padding, _mut_seq_rows_off_by_one,
-           _mut_batch_budget_of_next_sequence]
+           _mut_batch_budget_of_next_sequence, _mut_slots_misses_descending,
+           _mut_slots_refetch_hits]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)
