@@ -42,12 +42,13 @@ METRIC = "chunked-prefill sparse-attn tokens/s (select+attend) and % of roofline
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 def launches_per_step(w):
-    """Kernels one step launches.  Selection: query subselect, scoring and top-k, or only
-    scoring and top-k when every query is kept and G * C <= 16 (the decode shape).
+    """Kernels one step launches.  Selection: query subselect (or, when every query is kept
+    and G * C <= 16, the decode shape, the kept queries' operand block for bf16 and nothing
+    for fp32), scoring and top-k.
     Attention: the gather kernel and its combine when G * C <= 16, else compaction and
     the tensor-core kernel (bf16) or the CUDA-core kernel alone (fp32)."""
     small = w.group * w.chunk <= 16
-    sel = 2 if small and w.nq >= w.chunk else 3
+    sel = 3 if not (small and w.nq >= w.chunk) or w.dtype == "bf16" else 2
     att = 2 if small or w.dtype == "bf16" else 1
     return sel + att
 # DRAM traffic of one attention-kernel launch on the 128K-context workload
@@ -95,7 +96,8 @@ def stage_model(w: W.Workload):
     return st
 
 
-KERNEL_STAGE = {"qsub_kernel": "qsub", "score_tc_kernel": "score", "score_simt_kernel": "score",
+KERNEL_STAGE = {"qsub_kernel": "qsub", "kept_all_prep_kernel": "qsub", "score_tc_kernel": "score",
+                "score_tc2_kernel": "score", "score_simt_kernel": "score",
                 "score_decode_kernel": "score", "topk_kernel": "topk", "topk_block_kernel": "topk",
                 "attn_tc2_kernel": "attn", "attn_tc_kernel": "attn", "attn_simt_kernel": "attn",
                 "attn_decode_kernel": "attn"}
@@ -931,6 +933,201 @@ def run_perq(args):
     return 0
 
 
+# --------------------------------------------------------------------------------------
+# selected-value cache with miss-only fetch (decode steps with drifting queries)
+# --------------------------------------------------------------------------------------
+
+SELCACHE_METRIC = "decode steps over a selected-value cache with miss-only fetch, tokens/s, 1 B200"
+SELCACHE_SIGMA = 0.3       # per-step query drift (workloads.drifting_queries)
+
+
+def run_selcache(args):
+    from query_oriented_sparse_b200 import binding as Bd
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--selcache runs on one GPU")
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    base = W.WORKLOADS["decode_32"]
+    n_steps = args.warmup + args.steps + 1
+    w = W.custom("decode_32_drift", h_q=base.h_q, h_kv=base.h_kv, head_dim=base.head_dim, chunk=1,
+                 prefix=base.prefix, nq=1, budget=base.budget, recipe=base.recipe, seed=base.seed,
+                 prompt_chunks=n_steps)
+    t = W.generate(w)
+    qs = W.drifting_queries(base.seed + 100, t.q[:, :, 0], n_steps, SELCACHE_SIGMA).to(dev)
+    k, v = t.k_cache.to(dev), t.v_cache.to(dev)
+    b_max = max(w.budget)
+    shape = Bd.make_shape(w.batch, w.h_q, w.h_kv, w.head_dim, 1, w.torch_dtype)
+    ws = torch.empty(Bd.select_workspace_size(shape, max(w.prefix) + n_steps, w.nq),
+                     dtype=torch.uint8, device=dev)
+    aws = torch.empty(max(Bd.attn_workspace_size(shape, b_max), 256), dtype=torch.uint8, device=dev)
+    idx = torch.empty(w.batch, w.h_kv, b_max, dtype=torch.int32, device=dev)
+    out_p = torch.empty(w.batch, w.h_q, 1, w.head_dim, dtype=w.torch_dtype, device=dev)
+    out_c = torch.empty_like(out_p)
+    cache = Bd.SelCache(shape, b_max, dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    row_bytes = w.head_dim * w.elem_bytes
+    rec = {"plain_ms": [], "cache_ms": [], "misses": [], "selected": []}
+    for s in range(n_steps):
+        prefix = tuple(p + s for p in w.prefix)
+        q = qs[s]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        # plain: select, then the decode gather straight from the KV cache
+        flush.zero_()
+        ev[0].record(stream)
+        Bd.quoka_select(q, k, t.kv_off, prefix, w.nq, w.budget, b_max, idx_out=idx, workspace=ws)
+        Bd.sparse_chunk_attn(q, k, v, t.kv_off, prefix, w.budget, idx, out=out_p, workspace=aws)
+        ev[1].record(stream)
+        # cached: the same selection, the misses fetched into the cache, attention over it
+        flush.zero_()
+        ev[2].record(stream)
+        Bd.quoka_select(q, k, t.kv_off, prefix, w.nq, w.budget, b_max, idx_out=idx, workspace=ws)
+        misses = cache.update(k, v, t.kv_off, prefix, w.budget, idx)
+        cache.attend(q, prefix, w.budget, out=out_c)
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+        if s > args.warmup:                   # step 0 fills the empty cache
+            rec["plain_ms"].append(ev[0].elapsed_time(ev[1]))
+            rec["cache_ms"].append(ev[2].elapsed_time(ev[3]))
+            rec["misses"].append(int(misses.sum()))
+            rec["selected"].append(sum(w.h_kv * min(bb, p) for bb, p in zip(w.budget, prefix)))
+    assert Bd.device_error() == 0
+    o_p, o_c = out_p.float(), out_c.float()
+    err = float(((o_p - o_c).abs().amax(-1) / o_p.abs().amax(-1).clamp_min(1e-30)).max())
+    assert err <= 2e-2, f"cached attention differs from the plain path: {err}"
+    cache_ms = statistics.median(rec["cache_ms"])
+    plain_ms = statistics.median(rec["plain_ms"])
+    miss = sum(rec["misses"]) / max(sum(rec["selected"]), 1)
+    fetched = statistics.mean(rec["misses"]) * 2 * row_bytes + w.batch * w.h_kv * 2 * row_bytes
+    gathered = statistics.mean(rec["selected"]) * 2 * row_bytes
+    line = {
+        "metric": SELCACHE_METRIC, "value": w.batch / (cache_ms / 1e3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": cache_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": "decode_32_drift", "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
+                   "head_dim": w.head_dim, "prefix": "decode_32's, growing one row per step",
+                   "budget": list(w.budget), "query_drift_sigma": SELCACHE_SIGMA,
+                   "l2": "256 MB flush before every timed step of each arm",
+                   "launch": "eager (the prefix grows every step)"},
+        "gpu_launches": 11 * args.steps,    # 4 plain + 7 cached (select 2, update 2, attend 3)
+        "plain_tokens_per_s": w.batch / (plain_ms / 1e3), "plain_ms_per_step": plain_ms,
+        "miss_fraction": miss,
+        "fetched_bytes_per_step": fetched,
+        "plain_gathered_bytes_per_step": gathered,
+        "max_rel_diff_vs_plain": err,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+PERQ_TC_S = 2048           # keys per query token
+PERQ_TC_GROUP = 64         # consecutive tokens drawing from one base set
+PERQ_TC_SHARED = 0.9       # fraction of a token's set taken from its run's base set
+
+
+def perq_tc_unions(sel_kv, tp):
+    """Union size of every pair tile (2 * tp consecutive tokens of a KV head) for token
+    sets sel_kv int32 [h_kv, C, S] that every head of the group shares."""
+    h_kv, C, S = sel_kv.shape
+    out = []
+    for g in range(h_kv):
+        for t0 in range(0, C, 2 * tp):
+            out.append(int(torch.unique(sel_kv[g, t0:t0 + 2 * tp]).numel()))
+    return out
+
+
+def run_perq_tc(args):
+    from query_oriented_sparse_b200 import binding as Bd
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--perq-tc runs on one GPU")
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks, peak_src = load_peaks()
+    w = W.WORKLOADS["ctx_128k"]
+    t = W.generate(w)
+    n_rows = t.kv_off[1]
+    G = w.group
+    # one set per token and KV head, read by every query head of the group (causal)
+    sel_kv = W.per_query_selection_large(11, w.h_kv, w.chunk, n_rows, PERQ_TC_S, group=PERQ_TC_GROUP,
+                                         shared=PERQ_TC_SHARED, causal_prefix=w.prefix[0])
+    tp = 128 // G
+    unions = perq_tc_unions(sel_kv, tp)
+    cap = (max(unions) + 127) // 128 * 128
+    sel = sel_kv[:, None].expand(w.h_kv, G, w.chunk, PERQ_TC_S).reshape(1, w.h_q, w.chunk, PERQ_TC_S)
+    sel = sel.contiguous().to(dev)
+    q, k, v = t.q.to(dev), t.k_cache.to(dev), t.v_cache.to(dev)
+    shape = Bd.shape_of(q, k)
+    ws_tc = torch.empty(Bd.perq_tc_workspace_size(shape, PERQ_TC_S, cap), dtype=torch.uint8, device=dev)
+    ws_cc = torch.empty(Bd.perq_workspace_size(shape, PERQ_TC_S), dtype=torch.uint8, device=dev)
+    out_tc, out_cc = torch.empty_like(q), torch.empty_like(q)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call_tc():
+        Bd.sparse_perq_attn_tc(q, k, v, t.kv_off, sel, cap, out=out_tc, workspace=ws_tc)
+
+    def call_cc():
+        Bd.sparse_perq_attn(q, k, v, t.kv_off, sel, out=out_cc, workspace=ws_cc)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        return statistics.median(ms)
+
+    with ClockSampler(0) as clk:
+        tc_ms = timed(call_tc)
+    cc_ms = timed(call_cc)
+    assert Bd.device_error() == 0
+    o1, o2 = out_tc.float(), out_cc.float()
+    diff = float(((o1 - o2).abs().amax(-1) / o2.abs().amax(-1).clamp_min(1e-30)).max())
+    assert diff <= 2e-2, f"the two per-query forms differ: {diff}"
+    with Bd.KernelTimer(stream=stream) as kt:
+        call_tc()
+    kernels = {name: ms * 1e3 for name, ms in kt.times}
+    flops_union = 4.0 * w.head_dim * 256 * sum(unions)         # dense MMAs over each tile's union
+    flops_useful = 4.0 * w.head_dim * w.h_q * w.chunk * PERQ_TC_S
+    attn_us = kernels.get("attn_tc2_kernel", tc_ms * 1e3)
+    a = flops_union / (attn_us / 1e6) / 1e12
+    line = {
+        "metric": "per-query sparse attention on tensor cores, tokens/s, 1 B200", "value": w.chunk / (tc_ms / 1e3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": tc_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "perq_tc_128k", "chunk": w.chunk, "cache_rows": n_rows, "h_q": w.h_q,
+                   "h_kv": w.h_kv, "head_dim": w.head_dim, "keys_per_token": PERQ_TC_S,
+                   "sets": "one per token and KV head, shared by the group's query heads",
+                   "locality_group": PERQ_TC_GROUP, "shared_fraction": PERQ_TC_SHARED, "causal": True,
+                   "pair_tile_rows": 256, "max_union": cap,
+                   "l2": "256 MB flush before every timed call", "launch": "eager"},
+        "gpu_launches": 3 * args.steps,
+        "union_keys_per_tile": {"mean": statistics.mean(unions), "max": max(unions)},
+        "cuda_core_form_ms": cc_ms, "speedup_vs_cuda_core_form": cc_ms / tc_ms,
+        "kernel_us": kernels,
+        "roofline": {"bound": "tensor", "achieved": a, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": a / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "attn_tc2_kernel (membership masks) over each pair tile's union",
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "flops_over_unions": flops_union, "flops_of_the_sets": flops_useful},
+        "max_rel_diff_vs_cuda_core_form": diff,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -945,7 +1142,19 @@ def main():
                     help="time a whole prompt through the prefill call (time to first token)")
     ap.add_argument("--perq", action="store_true",
                     help="time per-query sparse attention with shared loading")
+    ap.add_argument("--selcache", action="store_true",
+                    help="time decode steps over a selected-value cache with miss-only fetch")
+    ap.add_argument("--perq-tc", action="store_true",
+                    help="time per-query attention on tensor cores over 256-row pair tiles")
     args = ap.parse_args()
+    if args.perq_tc:
+        if args.impl != "ours":
+            raise SystemExit("--perq-tc has no reference arm")
+        return run_perq_tc(args)
+    if args.selcache:
+        if args.impl != "ours":
+            raise SystemExit("--selcache has no reference arm")
+        return run_selcache(args)
     if args.perq:
         if args.impl != "ours":
             raise SystemExit("--perq has no reference arm")

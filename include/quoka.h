@@ -195,6 +195,32 @@ quoka_status sparse_perq_attn(const quoka_shape* shape, const void* q_chunk,
 size_t sparse_perq_attn_workspace_size(const quoka_shape* shape, int S);
 
 /*
+ * sparse_perq_attn_tc - sparse_perq_attn on tensor cores, for sets that the rows of a
+ * tile largely share (QUILT page, summary: the shared entries are loaded once, and the
+ * sharing is organised to fit the accelerator's tiles).
+ *
+ * Same result and arguments as sparse_perq_attn (sel rows in any order, duplicates count
+ * once, -1 ignored, empty sets give zeros), computed per pair tile of 256 query rows: the
+ * G heads of a KV head at 2 x (128 / G) consecutive positions.  The tile's sets are merged
+ * into one union of keys (ascending), whose K/V rows are gathered once; dense 256-row
+ * tcgen05 MMAs compute the logits of every row against every union key, and a per-row
+ * membership mask keeps only the row's own keys in its softmax.  The work per tile grows
+ * with its union, so this pays when the union is a small multiple of S.
+ *   max_union   bound on any tile's union (1 .. about 40000, fixed by the masks' shared
+ *               memory); sizes the workspace.  A tile whose union is larger sets bit 3 of
+ *               the device error word and keeps only its first max_union keys (that
+ *               tile's result is then wrong).
+ *   workspace   sparse_perq_attn_tc_workspace_size(shape, S, max_union) bytes
+ * Limits: bf16, head_dim 128, sequences of 1 .. 262144 rows.  Errors: INVALID_ARG,
+ * UNSUPPORTED, WORKSPACE, CUDA.
+ */
+quoka_status sparse_perq_attn_tc(const quoka_shape* shape, const void* q_chunk,
+                                 const void* k_cache, const void* v_cache,
+                                 const int64_t* kv_off, const int32_t* sel, int S, int max_union,
+                                 void* out, void* workspace, size_t ws_bytes, void* stream);
+size_t sparse_perq_attn_tc_workspace_size(const quoka_shape* shape, int S, int max_union);
+
+/*
  * quoka_step - one step of a chunked prefill or of decode, the way a serving loop runs
  * it: the chunk's new K/V rows go into the cache inside the call, then quoka_select and
  * sparse_chunk_attn run as described above (QUOKA page, Figure 1(a): each chunk sub-
@@ -273,6 +299,59 @@ quoka_status quoka_prefill(const quoka_shape* shape, int n_chunks, const void* q
 size_t quoka_prefill_workspace_size(const quoka_shape* shape, int n_chunks, int nq, int b_max);
 
 /*
+ * Selected-value cache with miss-only fetch (SQD page, the paragraph on sparse
+ * attention: the top-k choice still scans the whole cache where the cache lives, and
+ * attention over the chosen positions runs elsewhere; the chosen values are kept there
+ * and only the misses are sent, ahead of time).
+ *
+ * The cache keeps, per (sequence, KV head), the K/V rows of the current selection in a
+ * block laid out as the attention kernels read it: `kc_rows` = (b_max + chunk) rounded
+ * up to a multiple of 128 rows; slots 0 .. n-1 (n = min(budget[b], prefix_len[b])) hold
+ * the selected prefix rows in slot order, slots n .. n+chunk-1 the chunk's own rows
+ * (cache rows prefix_len[b] + t), then zero rows up to the next multiple of 128.
+ *   sel_cache  device, caller-owned, quoka_selcache_bytes() bytes, 256-byte aligned:
+ *              all K blocks [batch][h_kv][kc_rows][head_dim], then all V blocks, in
+ *              the shape's dtype.
+ *   slot_rows  device int32 [batch][h_kv][b_max], caller-owned: the row (relative to
+ *              the sequence's kv_off) that each slot holds, -1 for none.  Fill it with
+ *              -1 before the first update; afterwards only the updates write it.
+ * One cache serves one shape (batch, h_kv, head_dim, chunk, dtype) and one b_max.
+ *
+ * quoka_selcache_update - bring the cache to a new selection `idx` (as quoka_select
+ * writes it: [batch][h_kv][b_max], n ascending rows < prefix_len[b], then -1).  A row
+ * the cache already holds in a slot below n stays in that slot (a hit: no copy); the
+ * rows it does not hold (the misses) are copied from k_cache / v_cache into the slots
+ * that fell free, the k-th miss in ascending row order into the k-th free slot in
+ * ascending slot order; slots at or past n are emptied; the chunk rows and the zero
+ * rows are rewritten.  `misses` (device int32 [batch][h_kv], or NULL) receives the
+ * number of rows fetched per (sequence, KV head).  Arguments as for quoka_select; the
+ * workspace (quoka_selcache_workspace_size() bytes) is scratch.  The longest prefix and
+ * b_max must fit one shared-memory bitmap each (prefix + b_max up to about 900K rows);
+ * longer calls return QUOKA_ERR_UNSUPPORTED.  Asynchronous on `stream`; an index outside
+ * [0, prefix_len) sets the device error word (quoka_device_error) and is skipped.
+ *
+ * sparse_chunk_attn_selcache - the attention of sparse_chunk_attn, reading the selected
+ * and the chunk's K/V rows from the cache instead of gathering them from the KV cache:
+ * query t of head h attends to the n slots of KV head h / G and to chunk slots n .. n+t.
+ * The result is the attention over the set of rows the slots hold; it is bit-identical
+ * to sparse_chunk_attn over the same selection when the slots hold the rows in ascending
+ * order (after an update from an empty cache, or one with no miss from such a state), and
+ * equal up to the order of floating-point summation otherwise.  The workspace is the
+ * same size as the update's.
+ */
+size_t quoka_selcache_bytes(const quoka_shape* shape, int b_max);
+size_t quoka_selcache_workspace_size(const quoka_shape* shape, int b_max);
+quoka_status quoka_selcache_update(const quoka_shape* shape, const void* k_cache, const void* v_cache,
+                                   const int64_t* kv_off, const int32_t* prefix_len,
+                                   const int32_t* budget, const int32_t* idx, int b_max,
+                                   void* sel_cache, int32_t* slot_rows, int32_t* misses,
+                                   void* workspace, size_t ws_bytes, void* stream);
+quoka_status sparse_chunk_attn_selcache(const quoka_shape* shape, const void* q_chunk,
+                                        const int32_t* prefix_len, const int32_t* budget,
+                                        const void* sel_cache, int b_max, void* out,
+                                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * quoka_select_noalloc - quoka_select without a caller-provided workspace.
  *
  * The paper has no counterpart to this call; it exists for callers that cannot
@@ -327,7 +406,8 @@ int quoka_profile_marks(const char** names, int max_names);
 const char* quoka_last_error(void);
 
 /*
- * Reads and clears the device error word (0 = no kernel gave up a bounded wait).
+ * Reads and clears the device error word (0 = none): bit 0 a bounded wait gave up, bit 2
+ * an index outside its range, bit 3 a per-query tile's union over max_union.
  * Synchronises `stream`.  Returns QUOKA_ERR_CUDA if the read itself fails.
  */
 quoka_status quoka_device_error(uint32_t* code, void* stream);

@@ -51,6 +51,9 @@ SIGNATURES = {
     "sparse_perq_attn": (ctypes.c_int, [_SHAPE_P, _P, _P, _P, _I64P, _P, ctypes.c_int, _P, _P,
                                         ctypes.c_size_t, _P]),
     "sparse_perq_attn_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int]),
+    "sparse_perq_attn_tc": (ctypes.c_int, [_SHAPE_P, _P, _P, _P, _I64P, _P, ctypes.c_int, ctypes.c_int,
+                                           _P, _P, ctypes.c_size_t, _P]),
+    "sparse_perq_attn_tc_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int, ctypes.c_int]),
     "quoka_step": (ctypes.c_int, [_SHAPE_P, _P, _P, _P, _P, _P, _I64P, _I32P, ctypes.c_int,
                                   _I32P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "quoka_step_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int, ctypes.c_int,
@@ -60,6 +63,12 @@ SIGNATURES = {
                                      ctypes.c_size_t, _P]),
     "quoka_prefill_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int, ctypes.c_int,
                                                        ctypes.c_int]),
+    "quoka_selcache_bytes": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int]),
+    "quoka_selcache_workspace_size": (ctypes.c_size_t, [_SHAPE_P, ctypes.c_int]),
+    "quoka_selcache_update": (ctypes.c_int, [_SHAPE_P, _P, _P, _I64P, _I32P, _I32P, _P, ctypes.c_int,
+                                             _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "sparse_chunk_attn_selcache": (ctypes.c_int, [_SHAPE_P, _P, _I32P, _I32P, _P, ctypes.c_int, _P,
+                                                  _P, ctypes.c_size_t, _P]),
     "quoka_profile_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     "quoka_profile_marks": (ctypes.c_int, [ctypes.POINTER(ctypes.c_char_p), ctypes.c_int]),
 }
@@ -239,6 +248,30 @@ def sparse_perq_attn(q_chunk: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
     return out
 
 
+def perq_tc_workspace_size(shape: QuokaShape, S: int, max_union: int) -> int:
+    return int(lib().sparse_perq_attn_tc_workspace_size(ctypes.byref(shape), int(S), int(max_union)))
+
+
+def sparse_perq_attn_tc(q_chunk: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                        kv_off: Sequence[int], sel: torch.Tensor, max_union: int,
+                        out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """sparse_perq_attn on tensor cores over 256-row pair tiles whose key unions hold at
+    most max_union keys; returns out [batch, h_q, C, d]."""
+    shape = shape_of(q_chunk, k_cache)
+    if out is None:
+        out = torch.empty_like(q_chunk)
+    S = int(sel.shape[-1])
+    if workspace is None:
+        n = perq_tc_workspace_size(shape, S, max_union)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q_chunk.device)
+    _check(lib().sparse_perq_attn_tc(
+        ctypes.byref(shape), _ptr(q_chunk), _ptr(k_cache), _ptr(v_cache), _host_i64(kv_off),
+        _ptr(sel), S, int(max_union), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream(stream))))
+    return out
+
+
 def step_workspace_size(shape: QuokaShape, max_prefix: int, nq: int, b_max: int) -> int:
     return int(lib().quoka_step_workspace_size(ctypes.byref(shape), int(max_prefix), int(nq),
                                                int(b_max)))
@@ -303,13 +336,69 @@ def device_error(stream: Optional[torch.cuda.Stream] = None) -> int:
     return code.value
 
 
+class SelCache:
+    """A selected-value cache (quoka_selcache_update / sparse_chunk_attn_selcache) for one
+    shape and b_max: the K/V blocks, the slot map (all -1 at first) and a workspace, all
+    torch device memory owned by this object."""
+
+    def __init__(self, shape: QuokaShape, b_max: int, device):
+        self.shape, self.b_max = shape, int(b_max)
+        n = int(lib().quoka_selcache_bytes(ctypes.byref(shape), self.b_max))
+        w = int(lib().quoka_selcache_workspace_size(ctypes.byref(shape), self.b_max))
+        if n == 0 or w == 0:
+            raise QuokaError(QUOKA_ERR_INVALID_ARG, "bad shape or b_max for a selected-value cache")
+        self.cache = torch.zeros(n, dtype=torch.uint8, device=device)
+        self.slot_rows = torch.full((shape.batch, shape.h_kv, self.b_max), -1, dtype=torch.int32,
+                                    device=device)
+        self.misses = torch.zeros(shape.batch, shape.h_kv, dtype=torch.int32, device=device)
+        self.workspace = torch.empty(w, dtype=torch.uint8, device=device)
+
+    def blocks(self, dtype: torch.dtype):
+        """(K, V) views [batch, h_kv, kc_rows, head_dim] of the cache."""
+        s = self.shape
+        half = self.cache.numel() // 2
+        esz = torch.empty((), dtype=dtype).element_size()
+        rows = (self.b_max + s.chunk + 127) // 128 * 128
+        n = s.batch * s.h_kv * rows * s.head_dim * esz
+        k = self.cache[:n].view(dtype).view(s.batch, s.h_kv, rows, s.head_dim)
+        v = self.cache[half:half + n].view(dtype).view(s.batch, s.h_kv, rows, s.head_dim)
+        return k, v
+
+    def update(self, k_cache: torch.Tensor, v_cache: torch.Tensor, kv_off: Sequence[int],
+               prefix_len: Sequence[int], budget: Sequence[int], idx: torch.Tensor,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """Brings the cache to the selection idx; returns the misses per (sequence, KV head)."""
+        if int(idx.shape[-1]) != self.b_max:
+            raise QuokaError(QUOKA_ERR_INVALID_ARG, "idx's last dimension must be the cache's b_max")
+        _check(lib().quoka_selcache_update(
+            ctypes.byref(self.shape), _ptr(k_cache), _ptr(v_cache), _host_i64(kv_off),
+            _host_i32(prefix_len), _host_i32(budget), _ptr(idx), self.b_max, _ptr(self.cache),
+            _ptr(self.slot_rows), _ptr(self.misses), _ptr(self.workspace),
+            self.workspace.numel(), ctypes.c_void_p(_stream(stream))))
+        return self.misses
+
+    def attend(self, q_chunk: torch.Tensor, prefix_len: Sequence[int], budget: Sequence[int],
+               out: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """sparse_chunk_attn over the cache's rows; returns out [batch, h_q, C, d]."""
+        if out is None:
+            out = torch.empty_like(q_chunk)
+        _check(lib().sparse_chunk_attn_selcache(
+            ctypes.byref(self.shape), _ptr(q_chunk), _host_i32(prefix_len), _host_i32(budget),
+            _ptr(self.cache), self.b_max, _ptr(out), _ptr(self.workspace), self.workspace.numel(),
+            ctypes.c_void_p(_stream(stream))))
+        return out
+
+
 class KernelTimer:
     """Per-kernel device times of the library calls made inside a ``with`` block.
 
-    Records a start event on the stream, hands the library a pool of timing events (one
-    is recorded after every kernel it launches from this thread, quoka_profile_events),
-    and afterwards yields (kernel name, milliseconds) pairs in launch order.  Eager calls
-    only: not inside a stream capture.
+    Enqueues a short spin kernel and a start event on the stream, hands the library a pool
+    of timing events (one is recorded after every kernel it launches from this thread,
+    quoka_profile_events), and afterwards yields (kernel name, milliseconds) pairs in
+    launch order.  The spin keeps the GPU busy while the host enqueues the calls, so each
+    gap between events is one kernel's device time.  Eager calls only: not inside a
+    stream capture.
     """
 
     def __init__(self, max_kernels: int = 64, stream: Optional[torch.cuda.Stream] = None):
@@ -323,6 +412,10 @@ class KernelTimer:
         self.times = []
 
     def __enter__(self):
+        # a spin kernel ahead of the calls keeps the GPU busy while the host enqueues them,
+        # so no host gap sits between the start event and the first kernel
+        with torch.cuda.stream(self.stream):
+            torch.cuda._sleep(4_000_000)
         self.start.record(self.stream)
         _check(lib().quoka_profile_events(self._handles, len(self.events)))
         return self

@@ -3,6 +3,10 @@
 // dense attention kernel; QUILT page: the K/V entries a group of queries selected in
 // common are loaded once and reused by all of them).
 //
+// The same kernel runs per-query selections (QUILT page, summary): each pair of CTAs then
+// attends over the union of its 256 rows' key sets, with a per-row membership mask in
+// place of the causal rule (perq_tc.cuh builds the union, the masks and the K/V block).
+//
 // A cluster of two CTAs on two SMs serves one (sequence, KV head, 2 x TP chunk
 // positions); CTA r owns query tile r: 128 rows packing the G query heads of the KV head
 // at TP = 128 / G positions, gathered once by TMA (tile::gather4).  The pair runs every
@@ -69,10 +73,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// kMember = false: the chunk step; block (b, g) of the compacted cache holds the n_b
+//   selected rows, then the chunk's rows, visible to position t up to its own.
+// kMember = true: per-query sets; block `tile` (one per pair of CTAs) holds the union of
+//   the tile's sets, ucount[tile] keys, and key u counts for a row when the row's mask
+//   word pair of u's 128-key block has u's bit (mask [tile][256 rows][mwords]).
+template <bool kMember>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT2_THREADS, 1)
 attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ SeqTable tab,
-                const __grid_constant__ Attn2Params p, __nv_bfloat16* __restrict__ out) {
+                const __grid_constant__ Attn2Params p, __nv_bfloat16* __restrict__ out,
+                const uint32_t* __restrict__ mask, const int32_t* __restrict__ ucount, int mwords) {
   using Cfg = At2Cfg;
   constexpr int D = Cfg::D;
   namespace cg = cooperative_groups;
@@ -102,11 +113,12 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
   const int npairs = (p.C + 2 * p.TP - 1) / (2 * p.TP);
   const int pair = npairs - 1 - (int)(blockIdx.x >> 1);     // longest key ranges first
   const int t0 = pair * 2 * p.TP;
-  const int nsel = tab.nsel[b];
+  const long long tile = ((long long)b * p.h_kv + g) * npairs + pair;
+  const int nsel = kMember ? 0 : tab.nsel[b];
   const int tend = min(p.C, t0 + 2 * p.TP);                  // positions [t0, tend) of the pair
-  const int nkeys = nsel + tend;
+  const int nkeys = kMember ? ucount[tile] : nsel + tend;
   const int nblk = (nkeys + 127) / 128;                      // same for both CTAs
-  const int kc_row0 = (int)((long long)(b * p.h_kv + g) * p.kc_stride);
+  const int kc_row0 = (int)(kMember ? tile * p.kc_stride : (long long)(b * p.h_kv + g) * p.kc_stride);
   constexpr uint16_t kBoth = 0x3;
 
   if (threadIdx.x == 0) {
@@ -259,6 +271,11 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     const int t = t0 + (int)rank * p.TP + r % p.TP;
     const bool row_valid = hl < p.G && t < p.C;
     const int tmin = t0 + (int)rank * p.TP;                 // smallest position in this tile
+    // membership words of this row and key half, block j at mrow_g[j * 4]
+    const uint32_t* mrow_g = kMember ? mask + ((size_t)tile * 256 + rank * 128 + r) * (size_t)mwords + half * 2
+                                     : nullptr;
+    uint2 mw_next = make_uint2(0u, 0u);
+    if (kMember && grp < nblk) mw_next = *reinterpret_cast<const uint2*>(mrow_g + grp * 4);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     int jlast = -1;
@@ -286,13 +303,23 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(u[i]);
       }
       ptx::tmem_ld_wait();
-      const int kb0 = j * 128 + half * 64;
-      if (kb0 + 63 >= nsel + tmin || kb0 + 63 >= nkeys) {   // keys reach the causal part
+      if constexpr (kMember) {
+        const uint2 mw = mw_next;                           // this block's words, loaded a block early
+        if (j + 2 < nblk) mw_next = *reinterpret_cast<const uint2*>(mrow_g + (j + 2) * 4);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const int kk = kb0 + c;
-          const bool valid = kk < nkeys && (kk < nsel || kk - nsel <= t);
-          if (!valid) s[c] = -INFINITY;
+          const uint32_t wv = c < 32 ? mw.x : mw.y;
+          if (!((wv >> (c & 31)) & 1u)) s[c] = -INFINITY;
+        }
+      } else {
+        const int kb0 = j * 128 + half * 64;
+        if (kb0 + 63 >= nsel + tmin || kb0 + 63 >= nkeys) {   // keys reach the causal part
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int kk = kb0 + c;
+            const bool valid = kk < nkeys && (kk < nsel || kk - nsel <= t);
+            if (!valid) s[c] = -INFINITY;
+          }
         }
       }
       float mx;

@@ -19,10 +19,11 @@ struct SeqTable {
   int nsel[QUOKA_MAX_BATCH];  // min(budget[b], prefix[b])
 };
 
-// Device error word: bit 0 = a bounded mbarrier wait gave up.
+// Device error word: bit 0 = a bounded wait gave up, bit 2 = an index outside its range,
+// bit 3 = a per-query tile's key union exceeded the caller's bound.
 __device__ unsigned int g_device_error;
 
-enum : unsigned int { ERR_WAIT_TIMEOUT = 1u, ERR_TMEM_ALLOC = 2u, ERR_BAD_INDEX = 4u };
+enum : unsigned int { ERR_WAIT_TIMEOUT = 1u, ERR_TMEM_ALLOC = 2u, ERR_BAD_INDEX = 4u, ERR_UNION_CAP = 8u };
 
 __device__ __forceinline__ void flag_error(unsigned int bit) { atomicOr(&g_device_error, bit); }
 

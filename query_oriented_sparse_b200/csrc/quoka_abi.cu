@@ -14,6 +14,7 @@
 #include "qsub.cuh"
 #include "score_simt.cuh"
 #include "score_tc.cuh"
+#include "score_tc2.cuh"
 #include "topk.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
@@ -22,6 +23,8 @@
 #include "attn_decode.cuh"
 #include "select_decode.cuh"
 #include "attn_perq.cuh"
+#include "selcache.cuh"
+#include "perq_tc.cuh"
 
 using namespace quoka;
 
@@ -132,6 +135,7 @@ struct WsLayout {
   int ncg, heads_per_cg;    // column groups per KV head for the tensor-core scoring
   bool tc;                  // tensor-core scoring (bf16) or CUDA-core scoring (fp32)
   bool dec;                 // every query kept and <= 16 rows per KV head: decode scoring
+  bool dec_pair;            // decode shapes scored by the SM-pair tensor-core kernel (bf16)
 };
 
 WsLayout ws_layout(const Dims& d, int max_prefix, int nq) {
@@ -140,7 +144,8 @@ WsLayout ws_layout(const Dims& d, int max_prefix, int nq) {
   w.nkp = (w.nk + 15) / 16 * 16;
   w.dec = w.nk == d.C && d.G * d.C <= ADC_MAX_ROWS;
   w.tc = !w.dec && d.dt == QUOKA_BF16 && w.nkp <= STC_SLICE;
-  if (w.tc) {
+  w.dec_pair = w.dec && d.dt == QUOKA_BF16 && ST2_SLICE % w.nkp == 0 && d.G * w.nkp <= ST2_MAXCOLS;
+  if (w.tc || w.dec_pair) {
     // a column group is at most two head-aligned slices of <= 256 columns
     const int hmax = 2 * (STC_SLICE / w.nkp);
     w.ncg = (d.G + hmax - 1) / hmax;
@@ -282,6 +287,50 @@ quoka_status launch_score_tc(const Dims& d, const SeqTable& tab, long long rows,
   return QUOKA_OK;
 }
 
+// The SM-pair form of the scoring: 256-key pair tiles, slices of 128 columns (whole heads:
+// the kept queries per head, padded to 16, divide 128).  Decode shapes use it (WsLayout's
+// dec_pair).
+template <int D>
+quoka_status launch_score_tc2(const Dims& d, const SeqTable& tab, long long rows, const void* k,
+                              unsigned char* ws, const WsLayout& w, cudaStream_t st) {
+  ScoreTcParams p;
+  p.h_kv = d.h_kv;
+  p.G = d.G;
+  p.nkp = w.nkp;
+  p.ncg = w.ncg;
+  p.heads_per_cg = w.heads_per_cg;
+  p.padded = w.nk < w.nkp ? 1 : 0;
+  p.rows_per_head = rows;
+  p.pooled_stride = w.pooled_stride;
+  p.cg_stride = w.cg_stride;
+  p.inv_G = 1.0f / (float)d.G;
+  long long units = 0;
+  for (int b = 0; b < d.batch; ++b) {
+    p.unit_base[b] = (int)units;
+    units += (long long)d.h_kv * w.ncg * ((tab.prefix[b] + ST2_PT - 1) / ST2_PT);
+  }
+  for (int b = d.batch; b <= QUOKA_MAX_BATCH; ++b) p.unit_base[b] = (int)units;
+  if (units == 0) return QUOKA_OK;
+  if (units >= (1ll << 31)) return fail(QUOKA_ERR_UNSUPPORTED, "too many key tiles");
+  p.total_units = (int)units;
+  CUtensorMap kmap, qmap;
+  quoka_status s;
+  if ((s = make_map_bf16(&kmap, k, (uint64_t)d.h_kv * rows, D, 64, 128, "k_cache")) != QUOKA_OK) return s;
+  if ((s = make_map_bf16(&qmap, ws + w.qsel, (uint64_t)d.batch * d.h_q * w.nkp, D, 64, ST2_QBOX,
+                         "kept queries")) != QUOKA_OK)
+    return s;
+  cudaError_t e;
+  const int smem = St2Cfg<D>::SMEM;
+  if ((e = ensure_smem(score_tc2_kernel<D>, smem)) != cudaSuccess) return cuda_fail(e, "score_tc2 smem");
+  const int clusters = (int)std::min<long long>(units, sm_count() / 2);
+  score_tc2_kernel<D><<<2 * clusters, ST2_THREADS, smem, st>>>(
+      kmap, qmap, tab, p, reinterpret_cast<const float*>(ws + w.qinv),
+      reinterpret_cast<const float*>(ws + w.qbias), reinterpret_cast<float*>(ws + w.pooled));
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score_tc2 launch");
+  prof_mark(st, "score_tc2_kernel");
+  return QUOKA_OK;
+}
+
 // Top-B per (sequence, KV head): one CTA per row when there are many rows short enough to
 // stage in shared memory, else a 16-CTA cluster per row.
 quoka_status launch_topk(const Dims& d, const SeqTable& tab, int b_max, int32_t* idx_out,
@@ -360,6 +409,19 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
   float* pooled = reinterpret_cast<float*>(ws + w.pooled);
   cudaError_t e;
 
+  if (w.dec_pair) {
+    if constexpr (sizeof(T) == 2) {
+      kept_all_prep_kernel<T, D><<<d.batch * d.h_q, 128, 0, st>>>(
+          reinterpret_cast<const T*>(q), d.C, w.nkp, nq, qsel, qinv, qbias, kept_out);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "kept_all_prep launch");
+      prof_mark(st, "kept_all_prep_kernel");
+      if (tab.max_prefix > 0) {
+        quoka_status s = launch_score_tc2<D>(d, tab, rows, k, ws, w, st);
+        if (s != QUOKA_OK) return s;
+      }
+      return launch_topk(d, tab, b_max, idx_out, w, pooled, st);
+    }
+  }
   if (w.dec) {
     quoka_status s = launch_select_decode<T, D>(d, tab, rows, q, k, nq, kept_out, pooled, w, st);
     if (s != QUOKA_OK) return s;
@@ -421,6 +483,10 @@ size_t attn_ws_bytes(const Dims& d, int b_max) {
 }
 
 template <int D>
+quoka_status launch_attn_tc_core(const Dims& d, const SeqTable& tab, const void* q, const void* kc,
+                                 const void* vc, long long kc_stride, void* out, cudaStream_t st);
+
+template <int D>
 quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                             const void* k, const void* v, const int32_t* idx, int b_max,
                             void* out, unsigned char* ws, cudaStream_t st,
@@ -450,6 +516,26 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "compact launch");
   prof_mark(st, "compact_kv_kernel");
   // 2. dense attention over it
+  return launch_attn_tc_core<D>(d, tab, q, kc, vc, p.kc_stride, out, st);
+}
+
+// The tensor-core attention over compacted blocks kc / vc of kc_stride rows per
+// (sequence, KV head): selected rows first, then the chunk rows, then zero rows.
+template <int D>
+quoka_status launch_attn_tc_core(const Dims& d, const SeqTable& tab, const void* q, const void* kc,
+                                 const void* vc, long long kc_stride, void* out, cudaStream_t st) {
+  AttnTcParams p;
+  p.h_q = d.h_q;
+  p.h_kv = d.h_kv;
+  p.G = d.G;
+  p.C = d.C;
+  p.TP = 128 / d.G;
+  p.b_max = 0;
+  p.kc_stride = kc_stride;
+  p.rows_per_head = 0;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  const size_t kc_rows = (size_t)d.batch * d.h_kv * kc_stride;
+  cudaError_t e;
   CUtensorMap qmap, kmap, vmap;
   quoka_status s;
   if ((s = make_map_bf16(&qmap, q, (uint64_t)d.batch * d.h_q * d.C, D, 64, 1, "q_chunk")) != QUOKA_OK) return s;
@@ -466,10 +552,11 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
     p2.kc_stride = p.kc_stride;
     p2.scale_log2 = p.scale_log2;
     const int smem2 = At2Cfg::SMEM;
-    if ((e = ensure_smem(attn_tc2_kernel, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
+    if ((e = ensure_smem(attn_tc2_kernel<false>, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
     dim3 grid2(2 * ((d.C + 2 * p.TP - 1) / (2 * p.TP)), d.h_kv, d.batch);
-    attn_tc2_kernel<<<grid2, AT2_THREADS, smem2, st>>>(qmap, kmap, vmap, tab, p2,
-                                                       reinterpret_cast<__nv_bfloat16*>(out));
+    attn_tc2_kernel<false><<<grid2, AT2_THREADS, smem2, st>>>(qmap, kmap, vmap, tab, p2,
+                                                              reinterpret_cast<__nv_bfloat16*>(out),
+                                                              nullptr, nullptr, 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_tc2 launch");
     prof_mark(st, "attn_tc2_kernel");
     return QUOKA_OK;
@@ -486,10 +573,12 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
   return QUOKA_OK;
 }
 
+// idx_stride: entries between the idx rows of consecutive (sequence, KV head) pairs
+// (b_max, or 0 when every pair reads the same list).
 template <typename T, int D, int R>
 quoka_status launch_attn_decode_r(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                                   const void* k, const void* v, const int32_t* idx, int b_max,
-                                  void* out, unsigned char* ws, cudaStream_t st) {
+                                  void* out, unsigned char* ws, cudaStream_t st, int idx_stride) {
   using Cfg = AdcCfg<T, D>;
   long long total = 0;
   int nmax = 0;
@@ -511,7 +600,7 @@ quoka_status launch_attn_decode_r(const Dims& d, const SeqTable& tab, long long 
   float* part = reinterpret_cast<float*>(ws);
   attn_decode_kernel<T, D, R><<<dim3(nsplit, d.h_kv, d.batch), Cfg::THREADS, smem, st>>>(
       reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(k), reinterpret_cast<const T*>(v),
-      rows, tab, d.h_q, d.h_kv, d.C, idx, b_max, (int)split, nsplit_ws, scale_log2, part);
+      rows, tab, d.h_q, d.h_kv, d.C, idx, idx_stride, (int)split, nsplit_ws, scale_log2, part);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode launch");
   prof_mark(st, "attn_decode_kernel");
   attn_decode_combine_kernel<T, D, R><<<dim3(d.h_kv, d.batch), 128, 0, st>>>(
@@ -524,13 +613,14 @@ quoka_status launch_attn_decode_r(const Dims& d, const SeqTable& tab, long long 
 template <typename T, int D>
 quoka_status launch_attn_decode(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                                 const void* k, const void* v, const int32_t* idx, int b_max,
-                                void* out, unsigned char* ws, cudaStream_t st) {
+                                void* out, unsigned char* ws, cudaStream_t st, int idx_stride = -1) {
+  const int is = idx_stride < 0 ? b_max : idx_stride;
   switch (decode_rows(d)) {
-    case 1: return launch_attn_decode_r<T, D, 1>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
-    case 2: return launch_attn_decode_r<T, D, 2>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
-    case 4: return launch_attn_decode_r<T, D, 4>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
-    case 8: return launch_attn_decode_r<T, D, 8>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
-    default: return launch_attn_decode_r<T, D, 16>(d, tab, rows, q, k, v, idx, b_max, out, ws, st);
+    case 1: return launch_attn_decode_r<T, D, 1>(d, tab, rows, q, k, v, idx, b_max, out, ws, st, is);
+    case 2: return launch_attn_decode_r<T, D, 2>(d, tab, rows, q, k, v, idx, b_max, out, ws, st, is);
+    case 4: return launch_attn_decode_r<T, D, 4>(d, tab, rows, q, k, v, idx, b_max, out, ws, st, is);
+    case 8: return launch_attn_decode_r<T, D, 8>(d, tab, rows, q, k, v, idx, b_max, out, ws, st, is);
+    default: return launch_attn_decode_r<T, D, 16>(d, tab, rows, q, k, v, idx, b_max, out, ws, st, is);
   }
 }
 
@@ -688,6 +778,175 @@ quoka_status run_prefill(const Dims& d, int n_chunks, const unsigned char* q, co
                        k_cache, v_cache, nq, b_max, idx, out + c * q_chunk, ws, aws, st);
     if (s != QUOKA_OK) return s;
   }
+  return QUOKA_OK;
+}
+
+
+// ---- selected-value cache ------------------------------------------------------------
+// The cache: K blocks then V blocks, each [batch * h_kv][kc_block_rows][d] in the dtype.
+size_t selcache_bytes(const Dims& d, int b_max) {
+  const size_t rows = (size_t)d.batch * d.h_kv * (size_t)kc_block_rows(d, b_max);
+  return 2 * align_up(rows * d.D * d.esz, 256);
+}
+
+struct SelWs {
+  size_t plan_slot, plan_row, plan_count, iota, part, total;
+};
+
+// One workspace serves both calls: the update's plan, the attention's slot list and
+// (decode shapes) split partials.
+SelWs selcache_ws(const Dims& d, int b_max) {
+  SelWs w;
+  const size_t nbg = (size_t)d.batch * d.h_kv;
+  size_t off = 0;
+  w.plan_slot = off;
+  off = align_up(off + nbg * b_max * 4, 256);
+  w.plan_row = off;
+  off = align_up(off + nbg * b_max * 4, 256);
+  w.plan_count = off;
+  off = align_up(off + nbg * 4, 256);
+  w.iota = off;
+  off = align_up(off + (size_t)b_max * 4, 256);
+  w.part = off;
+  off = align_up(off + (use_decode(d) ? attn_ws_bytes(d, b_max) : 0), 256);
+  w.total = off;
+  return w;
+}
+
+// Sequence table of the cache's own blocks for the gather kernels: block (b, g) starts
+// at row (b * h_kv + g) * stride, so the head stride is `stride` and sequence b starts at
+// b * h_kv * stride; the "prefix" is the n_b selected slots, the chunk rows follow them.
+SeqTable selcache_table(const Dims& d, const SeqTable& tab, long long stride) {
+  SeqTable t = tab;
+  t.max_prefix = 0;
+  for (int b = 0; b <= d.batch; ++b) t.kv_off[b] = (long long)b * d.h_kv * stride;
+  for (int b = 0; b < d.batch; ++b) {
+    t.prefix[b] = tab.nsel[b];
+    t.max_prefix = std::max(t.max_prefix, tab.nsel[b]);
+  }
+  return t;
+}
+
+template <typename T, int D>
+quoka_status launch_attn_selcache(const Dims& d, const SeqTable& tab, const void* q,
+                                  const unsigned char* cache, int b_max, void* out,
+                                  unsigned char* ws, const SelWs& sw, cudaStream_t st) {
+  const long long stride = kc_block_rows(d, b_max);
+  const unsigned char* kc = cache;
+  const unsigned char* vc = cache + selcache_bytes(d, b_max) / 2;
+  if (d.dt == QUOKA_BF16 && !use_decode(d))
+    return launch_attn_tc_core<D>(d, tab, q, kc, vc, stride, out, st);
+  cudaError_t e;
+  auto* iota = reinterpret_cast<int32_t*>(ws + sw.iota);
+  iota_kernel<<<(b_max + 255) / 256, 256, 0, st>>>(iota, b_max);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "iota launch");
+  prof_mark(st, "iota_kernel");
+  const SeqTable t2 = selcache_table(d, tab, stride);
+  const long long rows = (long long)d.batch * d.h_kv * stride;
+  if (use_decode(d))
+    return launch_attn_decode<T, D>(d, t2, stride, q, kc, vc, iota, b_max, out, ws + sw.part, st, 0);
+  const int s = attn_simt_smem_bytes<D>();
+  if ((e = ensure_smem(attn_simt_kernel<T, D>, s)) != cudaSuccess) return cuda_fail(e, "attn smem");
+  dim3 grid((d.C + ATS_ROWS - 1) / ATS_ROWS, d.h_q, d.batch);
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  (void)rows;
+  attn_simt_kernel<T, D><<<grid, ATS_THREADS, s, st>>>(
+      reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(kc), reinterpret_cast<const T*>(vc),
+      stride, t2, d.h_q, d.h_kv, d.C, iota, 0, reinterpret_cast<T*>(out), scale_log2);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn launch");
+  prof_mark(st, "attn_simt_kernel");
+  return QUOKA_OK;
+}
+
+template <int VPR>
+quoka_status launch_selcache_copy(const Dims& d, const SeqTable& tab, long long rows, const void* k,
+                                  const void* v, int b_max, unsigned char* cache, unsigned char* ws,
+                                  const SelWs& sw, cudaStream_t st) {
+  const long long stride = kc_block_rows(d, b_max);
+  const int nbg = d.batch * d.h_kv;
+  const int copiers = std::max(1, std::min(64, 2 * sm_count() / nbg));
+  selcache_copy_kernel<VPR><<<dim3(copiers, nbg), 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), rows, tab, d.h_kv, d.C,
+      b_max, stride, reinterpret_cast<const int32_t*>(ws + sw.plan_slot),
+      reinterpret_cast<const int32_t*>(ws + sw.plan_row), reinterpret_cast<const int32_t*>(ws + sw.plan_count),
+      reinterpret_cast<uint4*>(cache), reinterpret_cast<uint4*>(cache + selcache_bytes(d, b_max) / 2));
+  cudaError_t e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "selcache_copy launch");
+  prof_mark(st, "selcache_copy_kernel");
+  return QUOKA_OK;
+}
+
+// ---- per-query selections on tensor cores (pair tiles of 256 rows) ----------------------
+struct PerqTcPlan {
+  int TP, npt, tiles, cap, mwords;
+  long long stride;
+  size_t uni, ucount, mask, kc, vc, total;
+};
+
+PerqTcPlan perq_tc_plan(const Dims& d, int cap) {
+  PerqTcPlan p;
+  p.TP = 128 / d.G;
+  p.npt = (d.C + 2 * p.TP - 1) / (2 * p.TP);
+  p.tiles = d.batch * d.h_kv * p.npt;
+  p.cap = cap;
+  p.mwords = (cap + 127) / 128 * 4;
+  p.stride = (long long)align_up((size_t)cap, 128);
+  size_t off = 0;
+  p.uni = off;
+  off = align_up(off + (size_t)p.tiles * cap * 4, 256);
+  p.ucount = off;
+  off = align_up(off + (size_t)p.tiles * 4, 256);
+  p.mask = off;
+  off = align_up(off + (size_t)p.tiles * 256 * p.mwords * 4, 256);
+  p.kc = off;
+  off = align_up(off + (size_t)p.tiles * p.stride * d.D * 2, 256);
+  p.vc = off;
+  off = align_up(off + (size_t)p.tiles * p.stride * d.D * 2, 256);
+  p.total = off;
+  return p;
+}
+
+quoka_status launch_perq_tc(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                            const void* k, const void* v, const int32_t* sel, int S, void* out,
+                            unsigned char* ws, const PerqTcPlan& pl, cudaStream_t st) {
+  cudaError_t e;
+  auto* uni = reinterpret_cast<int32_t*>(ws + pl.uni);
+  auto* ucount = reinterpret_cast<int32_t*>(ws + pl.ucount);
+  auto* mask = reinterpret_cast<uint32_t*>(ws + pl.mask);
+  const int usmem = (int)perq_tc_union_smem(pl.cap);
+  if ((e = ensure_smem(perq_tc_union_kernel, usmem)) != cudaSuccess) return cuda_fail(e, "perq_tc_union smem");
+  perq_tc_union_kernel<<<dim3(pl.npt, d.h_kv, d.batch), PTC_THREADS, usmem, st>>>(
+      sel, tab, d.h_q, d.h_kv, d.C, S, pl.TP, pl.cap, uni, ucount, mask);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_tc_union launch");
+  prof_mark(st, "perq_tc_union_kernel");
+  const long long vecs = (long long)pl.tiles * pl.stride * 16;
+  const int grid = (int)std::min<long long>((vecs + 255) / 256, (long long)sm_count() * 16);
+  perq_tc_gather_kernel<16><<<grid, 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), rows, tab, d.h_kv, pl.npt,
+      pl.cap, pl.stride, uni, ucount, reinterpret_cast<uint4*>(ws + pl.kc), reinterpret_cast<uint4*>(ws + pl.vc),
+      vecs);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_tc_gather launch");
+  prof_mark(st, "perq_tc_gather_kernel");
+  CUtensorMap qmap, kmap, vmap;
+  quoka_status s;
+  const uint64_t kc_rows = (uint64_t)pl.tiles * pl.stride;
+  if ((s = make_map_bf16(&qmap, q, (uint64_t)d.batch * d.h_q * d.C, 128, 64, 1, "q_chunk")) != QUOKA_OK) return s;
+  if ((s = make_map_bf16(&kmap, ws + pl.kc, kc_rows, 128, 64, 64, "union K")) != QUOKA_OK) return s;
+  if ((s = make_map_bf16(&vmap, ws + pl.vc, kc_rows, 128, 64, 128, "union V")) != QUOKA_OK) return s;
+  Attn2Params p2;
+  p2.h_q = d.h_q;
+  p2.h_kv = d.h_kv;
+  p2.G = d.G;
+  p2.C = d.C;
+  p2.TP = pl.TP;
+  p2.kc_stride = pl.stride;
+  p2.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
+  const int smem2 = At2Cfg::SMEM;
+  if ((e = ensure_smem(attn_tc2_kernel<true>, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
+  attn_tc2_kernel<true><<<dim3(2 * pl.npt, d.h_kv, d.batch), AT2_THREADS, smem2, st>>>(
+      qmap, kmap, vmap, tab, p2, reinterpret_cast<__nv_bfloat16*>(out), mask, ucount, pl.mwords);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_tc2 (per-query) launch");
+  prof_mark(st, "attn_tc2_kernel");
   return QUOKA_OK;
 }
 
@@ -950,6 +1209,152 @@ quoka_status quoka_prefill(const quoka_shape* shape, int n_chunks, const void* q
                      : run_prefill<float, 128>(d, n_chunks, qb, kn, vn, k_cache, v_cache, kv_off, nq, budgets, b_max, idx, ob, ws, aws, st);
   return d.D == 64 ? run_prefill<__nv_bfloat16, 64>(d, n_chunks, qb, kn, vn, k_cache, v_cache, kv_off, nq, budgets, b_max, idx, ob, ws, aws, st)
                    : run_prefill<__nv_bfloat16, 128>(d, n_chunks, qb, kn, vn, k_cache, v_cache, kv_off, nq, budgets, b_max, idx, ob, ws, aws, st);
+}
+
+size_t sparse_perq_attn_tc_workspace_size(const quoka_shape* shape, int S, int max_union) {
+  Dims d;
+  if (check_shape(shape, &d) != QUOKA_OK || S < 1 || max_union < 1) return 0;
+  if (d.dt != QUOKA_BF16 || d.D != 128) return 0;
+  if (perq_tc_union_smem(max_union) > 227u * 1024u) return 0;
+  return perq_tc_plan(d, max_union).total;
+}
+
+quoka_status sparse_perq_attn_tc(const quoka_shape* shape, const void* q_chunk, const void* k_cache,
+                                 const void* v_cache, const int64_t* kv_off, const int32_t* sel, int S,
+                                 int max_union, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (d.dt != QUOKA_BF16 || d.D != 128)
+    return fail(QUOKA_ERR_UNSUPPORTED, "the tensor-core per-query attention takes bf16 with head_dim 128");
+  if (!q_chunk || !k_cache || !v_cache || !kv_off || !sel || !out)
+    return fail(QUOKA_ERR_INVALID_ARG, "q_chunk, k_cache, v_cache, kv_off, sel and out must be non-NULL");
+  if (!aligned(q_chunk, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(sel, 16) ||
+      !aligned(out, 16))
+    return fail(QUOKA_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (out == q_chunk || out == k_cache || out == v_cache)
+    return fail(QUOKA_ERR_INVALID_ARG, "out must not alias an input");
+  if (S < 1 || S > (1 << 20)) return fail(QUOKA_ERR_INVALID_ARG, "S must be in [1, 2^20] (got %d)", S);
+  if (max_union < 1) return fail(QUOKA_ERR_INVALID_ARG, "max_union must be >= 1 (got %d)", max_union);
+  if (perq_tc_union_smem(max_union) > 227u * 1024u)
+    return fail(QUOKA_ERR_UNSUPPORTED, "max_union %d is too large for one tile's masks", max_union);
+  if (kv_off[0] < 0) return fail(QUOKA_ERR_INVALID_ARG, "kv_off[0] must be >= 0");
+  SeqTable tab;
+  tab.batch = d.batch;
+  tab.max_prefix = 0;
+  for (int b = 0; b <= d.batch; ++b) tab.kv_off[b] = kv_off[b];
+  for (int b = d.batch + 1; b <= QUOKA_MAX_BATCH; ++b) tab.kv_off[b] = kv_off[d.batch];
+  for (int b = 0; b < QUOKA_MAX_BATCH; ++b) { tab.prefix[b] = 0; tab.nsel[b] = 0; }
+  for (int b = 0; b < d.batch; ++b) {
+    const long long n = kv_off[b + 1] - kv_off[b];
+    if (n < 1) return fail(QUOKA_ERR_INVALID_ARG, "sequence %d owns no cache rows", b);
+    if (n > (long long)PTC_MAX_WORDS * 32)
+      return fail(QUOKA_ERR_UNSUPPORTED, "sequence %d owns %lld rows; at most %d", b, n, PTC_MAX_WORDS * 32);
+  }
+  const PerqTcPlan pl = perq_tc_plan(d, max_union);
+  if ((long long)pl.tiles * pl.stride >= (1ll << 31))
+    return fail(QUOKA_ERR_UNSUPPORTED, "tiles x max_union too large");
+  if (!workspace) return fail(QUOKA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", pl.total);
+  if (!aligned(workspace, 256)) return fail(QUOKA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < pl.total) return fail(QUOKA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, pl.total);
+  return launch_perq_tc(d, tab, kv_off[d.batch], q_chunk, k_cache, v_cache, sel, S, out,
+                        reinterpret_cast<unsigned char*>(workspace), pl, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t quoka_selcache_bytes(const quoka_shape* shape, int b_max) {
+  Dims d;
+  if (check_shape(shape, &d) != QUOKA_OK || b_max < 1) return 0;
+  return selcache_bytes(d, b_max);
+}
+
+size_t quoka_selcache_workspace_size(const quoka_shape* shape, int b_max) {
+  Dims d;
+  if (check_shape(shape, &d) != QUOKA_OK || b_max < 1) return 0;
+  return selcache_ws(d, b_max).total;
+}
+
+quoka_status quoka_selcache_update(const quoka_shape* shape, const void* k_cache, const void* v_cache,
+                                   const int64_t* kv_off, const int32_t* prefix_len,
+                                   const int32_t* budget, const int32_t* idx, int b_max,
+                                   void* sel_cache, int32_t* slot_rows, int32_t* misses,
+                                   void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (!k_cache || !v_cache || !idx || !sel_cache || !slot_rows)
+    return fail(QUOKA_ERR_INVALID_ARG, "k_cache, v_cache, idx, sel_cache and slot_rows must be non-NULL");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(idx, 16) || !aligned(sel_cache, 256) ||
+      !aligned(slot_rows, 16) || (misses && !aligned(misses, 16)))
+    return fail(QUOKA_ERR_INVALID_ARG,
+                "device pointers must be 16-byte aligned (sel_cache 256-byte aligned)");
+  if (sel_cache == k_cache || sel_cache == v_cache)
+    return fail(QUOKA_ERR_INVALID_ARG, "sel_cache must not alias the cache");
+  SeqTable tab;
+  long long rows = 0;
+  if ((s = build_table(d, kv_off, prefix_len, budget, b_max, &tab, &rows)) != QUOKA_OK) return s;
+  const size_t smem = selcache_plan_smem(tab.max_prefix, b_max);
+  if (smem > 227u * 1024u)
+    return fail(QUOKA_ERR_UNSUPPORTED, "prefix %d with b_max %d is too long for the selected-value cache",
+                tab.max_prefix, b_max);
+  const SelWs sw = selcache_ws(d, b_max);
+  if (!workspace) return fail(QUOKA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", sw.total);
+  if (!aligned(workspace, 256)) return fail(QUOKA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < sw.total) return fail(QUOKA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, sw.total);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* ws = reinterpret_cast<unsigned char*>(workspace);
+  cudaError_t e;
+  if ((e = ensure_smem(selcache_plan_kernel, (int)smem)) != cudaSuccess) return cuda_fail(e, "selcache_plan smem");
+  selcache_plan_kernel<<<dim3(d.h_kv, d.batch), SCP_THREADS, smem, st>>>(
+      tab, d.h_kv, b_max, idx, slot_rows, reinterpret_cast<int32_t*>(ws + sw.plan_slot),
+      reinterpret_cast<int32_t*>(ws + sw.plan_row), reinterpret_cast<int32_t*>(ws + sw.plan_count), misses);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "selcache_plan launch");
+  prof_mark(st, "selcache_plan_kernel");
+  auto* cache = reinterpret_cast<unsigned char*>(sel_cache);
+  switch (d.D * d.esz / 16) {
+    case 8: return launch_selcache_copy<8>(d, tab, rows, k_cache, v_cache, b_max, cache, ws, sw, st);
+    case 16: return launch_selcache_copy<16>(d, tab, rows, k_cache, v_cache, b_max, cache, ws, sw, st);
+    default: return launch_selcache_copy<32>(d, tab, rows, k_cache, v_cache, b_max, cache, ws, sw, st);
+  }
+}
+
+quoka_status sparse_chunk_attn_selcache(const quoka_shape* shape, const void* q_chunk,
+                                        const int32_t* prefix_len, const int32_t* budget,
+                                        const void* sel_cache, int b_max, void* out,
+                                        void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  quoka_status s = check_shape(shape, &d);
+  if (s != QUOKA_OK) return s;
+  if (!q_chunk || !sel_cache || !out || !prefix_len || !budget)
+    return fail(QUOKA_ERR_INVALID_ARG, "q_chunk, prefix_len, budget, sel_cache and out must be non-NULL");
+  if (!aligned(q_chunk, 16) || !aligned(sel_cache, 256) || !aligned(out, 16))
+    return fail(QUOKA_ERR_INVALID_ARG, "device pointers must be 16-byte aligned (sel_cache 256-byte aligned)");
+  if (out == q_chunk || out == sel_cache) return fail(QUOKA_ERR_INVALID_ARG, "out must not alias an input");
+  if (b_max < 1) return fail(QUOKA_ERR_INVALID_ARG, "b_max must be >= 1 (got %d)", b_max);
+  SeqTable tab;
+  tab.batch = d.batch;
+  tab.max_prefix = 0;
+  for (int b = 0; b <= QUOKA_MAX_BATCH; ++b) tab.kv_off[b] = 0;
+  for (int b = 0; b < QUOKA_MAX_BATCH; ++b) { tab.prefix[b] = 0; tab.nsel[b] = 0; }
+  for (int b = 0; b < d.batch; ++b) {
+    if (prefix_len[b] < 0) return fail(QUOKA_ERR_INVALID_ARG, "prefix_len[%d] = %d < 0", b, prefix_len[b]);
+    if (budget[b] < 0 || budget[b] > b_max)
+      return fail(QUOKA_ERR_INVALID_ARG, "budget[%d] = %d outside [0, b_max=%d]", b, budget[b], b_max);
+    tab.prefix[b] = prefix_len[b];
+    tab.nsel[b] = std::min(budget[b], prefix_len[b]);
+    tab.max_prefix = std::max(tab.max_prefix, prefix_len[b]);
+  }
+  const SelWs sw = selcache_ws(d, b_max);
+  if (!workspace) return fail(QUOKA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", sw.total);
+  if (!aligned(workspace, 256)) return fail(QUOKA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < sw.total) return fail(QUOKA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, sw.total);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* ws = reinterpret_cast<unsigned char*>(workspace);
+  const auto* cache = reinterpret_cast<const unsigned char*>(sel_cache);
+  if (d.dt == QUOKA_F32)
+    return d.D == 64 ? launch_attn_selcache<float, 64>(d, tab, q_chunk, cache, b_max, out, ws, sw, st)
+                     : launch_attn_selcache<float, 128>(d, tab, q_chunk, cache, b_max, out, ws, sw, st);
+  return d.D == 64 ? launch_attn_selcache<__nv_bfloat16, 64>(d, tab, q_chunk, cache, b_max, out, ws, sw, st)
+                   : launch_attn_selcache<__nv_bfloat16, 128>(d, tab, q_chunk, cache, b_max, out, ws, sw, st);
 }
 
 }  // extern "C"

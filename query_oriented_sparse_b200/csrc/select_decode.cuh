@@ -19,6 +19,7 @@
 //                        cluster_select.cuh with block barriers only.
 #pragma once
 #include "cluster_select.cuh"
+#include "tc_ptx.cuh"
 
 namespace quoka {
 
@@ -77,6 +78,49 @@ __device__ __forceinline__ void scd_vec16(const unsigned char* p, float (&x)[16 
       x[2 * i] = f.x; x[2 * i + 1] = f.y;
     }
   }
+}
+
+// Every query kept (decode shapes) and the scoring on tensor cores: the operand block of
+// the kept queries without a subselect.  One CTA per (sequence, query head): row t < C is
+// query t (raw), its 1/|q| (0 for a zero query) and bias 0; rows C .. nkp-1 are zero with
+// bias -inf, so they never win a max; kept_out (if asked) lists 0 .. C-1, then -1.
+template <typename T, int D>
+__global__ void __launch_bounds__(128)
+kept_all_prep_kernel(const T* __restrict__ q, int C, int nkp, int nq, T* __restrict__ qsel,
+                     float* __restrict__ qinv, float* __restrict__ qbias, int32_t* __restrict__ kept_out) {
+  constexpr int VPR = D * (int)sizeof(T) / 16;
+  const int bh = blockIdx.x;                   // b * h_q + h, row block bh * nkp
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = warp; t < nkp; t += 4) {
+    const size_t row = (size_t)bh * nkp + t;
+    uint4* dst = reinterpret_cast<uint4*>(qsel + row * D);
+    if (t < C) {
+      const uint4* src = reinterpret_cast<const uint4*>(q + ((size_t)bh * C + t) * D);
+      float ss = 0.f;
+      for (int v = lane; v < VPR; v += 32) {
+        const uint4 x = __ldg(src + v);
+        dst[v] = x;
+        float f[16 / sizeof(T)];
+        scd_vec16<T>(reinterpret_cast<const unsigned char*>(&x), f);
+#pragma unroll
+        for (int e = 0; e < (int)(16 / sizeof(T)); ++e) ss = fmaf(f[e], f[e], ss);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) {
+        qinv[row] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+        qbias[row] = 0.f;
+      }
+    } else {
+      for (int v = lane; v < VPR; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+      if (lane == 0) {
+        qinv[row] = 0.f;
+        qbias[row] = -INFINITY;
+      }
+    }
+  }
+  if (kept_out)
+    for (int i = threadIdx.x; i < nq; i += blockDim.x) kept_out[(size_t)bh * nq + i] = i < C ? i : -1;
 }
 
 // Rows r = j * C + t of a KV head: query head g*G + j, chunk position t (all kept).
@@ -147,25 +191,50 @@ score_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, long long 
     __syncwarp();
     const unsigned char* krow = stage + (bt & 1) * Cfg::STAGE + lane * ROW;
     float dot[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) dot[r] = 0.f;
     float nn = 0.f;
+    if constexpr (sizeof(T) == 2) {
+      // bf16 keys: even and odd dimensions in the two halves of packed fp32x2 FMAs
+      float2 dot2[R], nn2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < R; ++r) dot2[r] = make_float2(0.f, 0.f);
 #pragma unroll 2
-    for (int c = 0; c < VPR; ++c) {
-      float kx[EPV];
-      scd_vec16<T>(krow + c * 16, kx);
+      for (int c = 0; c < VPR; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(krow + c * 16);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < EPV; ++e) nn = fmaf(kx[e], kx[e], nn);
+        for (int i = 0; i < 4; ++i) {
+          const float2 k2 = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+          nn2 = ptx::fma2(k2, k2, nn2);
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float* qr = qs + r * D + c * EPV;
+          for (int r = 0; r < R; ++r) {
+            const float2 q2 = *reinterpret_cast<const float2*>(qs + r * D + c * EPV + 2 * i);
+            dot2[r] = ptx::fma2(q2, k2, dot2[r]);
+          }
+        }
+      }
 #pragma unroll
-        for (int e4 = 0; e4 < EPV; e4 += 4) {
-          const float4 qv = *reinterpret_cast<const float4*>(qr + e4);
-          dot[r] = fmaf(qv.x, kx[e4], dot[r]);
-          dot[r] = fmaf(qv.y, kx[e4 + 1], dot[r]);
-          dot[r] = fmaf(qv.z, kx[e4 + 2], dot[r]);
-          dot[r] = fmaf(qv.w, kx[e4 + 3], dot[r]);
+      for (int r = 0; r < R; ++r) dot[r] = dot2[r].x + dot2[r].y;
+      nn = nn2.x + nn2.y;
+    } else {
+#pragma unroll
+      for (int r = 0; r < R; ++r) dot[r] = 0.f;
+#pragma unroll 2
+      for (int c = 0; c < VPR; ++c) {
+        float kx[EPV];
+        scd_vec16<T>(krow + c * 16, kx);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) nn = fmaf(kx[e], kx[e], nn);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const float* qr = qs + r * D + c * EPV;
+#pragma unroll
+          for (int e4 = 0; e4 < EPV; e4 += 4) {
+            const float4 qv = *reinterpret_cast<const float4*>(qr + e4);
+            dot[r] = fmaf(qv.x, kx[e4], dot[r]);
+            dot[r] = fmaf(qv.y, kx[e4 + 1], dot[r]);
+            dot[r] = fmaf(qv.z, kx[e4 + 2], dot[r]);
+            dot[r] = fmaf(qv.w, kx[e4 + 3], dot[r]);
+          }
         }
       }
     }

@@ -162,6 +162,15 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, u
       "r"(r2), "r"(r3)
       : "memory");
 }
+// Contiguous global->shared copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) whose completion is counted on this CTA's mbarrier.  No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 // 16-byte asynchronous global->shared copy (L2 only), and the arrival on an mbarrier
 // once every copy issued so far by this thread has landed (does not add to the
 // barrier's expected count, so the barrier is initialised with one count per thread).

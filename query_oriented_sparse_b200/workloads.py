@@ -272,3 +272,19 @@ def per_query_selection_large(seed: int, h_q: int, n_queries: int, n_keys: int, 
         rows = torch.where(take, base[gid], own)
         out[h] = torch.sort(rows, dim=1).values.to(torch.int32)
     return out
+
+
+def drifting_queries(seed: int, q0: torch.Tensor, steps: int, sigma: float = 0.3) -> torch.Tensor:
+    """Queries of consecutive decode steps that drift: step 0 is q0 [batch, h_q, d]; step
+    s adds sigma * |q_{s-1}| / sqrt(d) * N(0, I) to step s-1's query (per row), so
+    consecutive steps point in nearby directions and select overlapping key sets, as
+    consecutive tokens of one text do.  Returns [steps, batch, h_q, 1, d] in q0's dtype."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    d = q0.shape[-1]
+    cur = q0.float()
+    out = [cur]
+    for _ in range(1, steps):
+        noise = torch.randn(cur.shape, generator=g)
+        cur = cur + sigma * cur.norm(dim=-1, keepdim=True) / math.sqrt(d) * noise
+        out.append(cur)
+    return torch.stack(out, 0).unsqueeze(-2).to(q0.dtype).contiguous()

@@ -231,3 +231,73 @@ def test_profile_events_host_checks():
     assert lib.quoka_profile_events(empty, 1) == Bd.QUOKA_ERR_INVALID_ARG
     assert lib.quoka_profile_events(empty, 0) == Bd.QUOKA_ERR_INVALID_ARG
     assert lib.quoka_profile_marks(None, 0) == 0
+
+
+def test_selcache_sizes():
+    s = Bd.make_shape(2, 8, 2, 128, 96, torch.bfloat16)
+    lib = Bd.lib()
+    # K and V blocks of 2 x 2 (sequence, KV head) pairs x (200 + 96 -> 384 rows) x 256 B
+    assert lib.quoka_selcache_bytes(ctypes.byref(s), 200) == 2 * 4 * 384 * 256
+    assert lib.quoka_selcache_workspace_size(ctypes.byref(s), 200) > 2 * 4 * 200 * 4
+    assert lib.quoka_selcache_bytes(ctypes.byref(s), 0) == 0
+    bad = Bd.make_shape(1, 8, 2, 96, 96, torch.bfloat16)
+    assert lib.quoka_selcache_bytes(ctypes.byref(bad), 64) == 0
+
+
+def _selupd(shape, k=FAKE, v=FAKE + 0x1000, kv_off=(0, 1024), prefix=(512,), budget=(64,),
+            idx=FAKE + 0x2000, b_max=64, cache=FAKE + 0x10000, slots=FAKE + 0x3000, misses=None,
+            ws=FAKE + 0x4000, ws_bytes=1 << 30):
+    return Bd.lib().quoka_selcache_update(
+        ctypes.byref(shape), k, v, Bd._host_i64(kv_off), Bd._host_i32(prefix), Bd._host_i32(budget),
+        idx, b_max, cache, slots, misses, ws, ws_bytes, None)
+
+
+@no_gpu
+@pytest.mark.parametrize("case,status", [
+    (dict(shape=dict(head_dim=96)), Bd.QUOKA_ERR_UNSUPPORTED),
+    (dict(idx=None), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(slots=None), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(cache=FAKE + 0x10010), Bd.QUOKA_ERR_INVALID_ARG),   # not 256-byte aligned
+    (dict(cache=FAKE), Bd.QUOKA_ERR_INVALID_ARG),             # aliases k_cache
+    (dict(budget=(65,)), Bd.QUOKA_ERR_INVALID_ARG),
+    (dict(prefix=(1000,)), Bd.QUOKA_ERR_INVALID_ARG),         # prefix + chunk > rows
+    (dict(ws=None), Bd.QUOKA_ERR_WORKSPACE),
+    (dict(ws_bytes=64), Bd.QUOKA_ERR_WORKSPACE),
+    (dict(kv_off=(0, 1 << 21), prefix=(1 << 21) - 300, b_max=1 << 19, budget=(1 << 19,)),
+     Bd.QUOKA_ERR_UNSUPPORTED),                                # bitmaps beyond shared memory
+])
+def test_selcache_update_rejects(case, status):
+    shp = dict(batch=1, h_q=8, h_kv=2, head_dim=128, chunk=256, dtype=Bd.QUOKA_BF16)
+    shp.update(case.pop("shape", {}))
+    if isinstance(case.get("prefix"), int):
+        case["prefix"] = (case["prefix"],)
+    assert _selupd(Bd.QuokaShape(**shp), **case) == status
+
+
+@no_gpu
+def test_selcache_attn_rejects():
+    lib = Bd.lib()
+    s = Bd.QuokaShape(1, 8, 2, 128, 256, Bd.QUOKA_BF16)
+
+    def call(q=FAKE, budget=(64,), cache=FAKE + 0x10000, b_max=64, out=FAKE + 0x20000, ws=FAKE + 0x30000,
+             ws_bytes=1 << 30):
+        return lib.sparse_chunk_attn_selcache(ctypes.byref(s), q, Bd._host_i32((512,)), Bd._host_i32(budget),
+                                              cache, b_max, out, ws, ws_bytes, None)
+    assert call(out=FAKE) == Bd.QUOKA_ERR_INVALID_ARG            # aliases q
+    assert call(budget=(65,)) == Bd.QUOKA_ERR_INVALID_ARG
+    assert call(b_max=0, budget=(0,)) == Bd.QUOKA_ERR_INVALID_ARG
+    assert call(cache=FAKE + 0x10008) == Bd.QUOKA_ERR_INVALID_ARG
+    assert call(ws=None) == Bd.QUOKA_ERR_WORKSPACE
+    assert call(ws_bytes=16) == Bd.QUOKA_ERR_WORKSPACE
+
+
+def test_perq_tc_sizes_and_limits():
+    lib = Bd.lib()
+    s = Bd.make_shape(1, 32, 8, 128, 4096, torch.bfloat16)
+    n = lib.sparse_perq_attn_tc_workspace_size(ctypes.byref(s), 512, 8192)
+    # 8 KV heads x 64 pair tiles: union K/V blocks of 8192 rows of 256 B each, plus masks
+    tiles = 8 * 64
+    assert n >= tiles * 8192 * 256 * 2 + tiles * 256 * (8192 // 32) * 4
+    assert lib.sparse_perq_attn_tc_workspace_size(ctypes.byref(s), 512, 1 << 20) == 0   # masks too large
+    f32 = Bd.make_shape(1, 32, 8, 128, 4096, torch.float32)
+    assert lib.sparse_perq_attn_tc_workspace_size(ctypes.byref(f32), 512, 8192) == 0

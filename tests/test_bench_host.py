@@ -130,3 +130,10 @@ def test_kernel_table_per_launch_rooflines():
     # a kernel launched twice per step is reported per launch
     tab2 = bench.kernel_table(w, [[("qsub_kernel", 0.01), ("qsub_kernel", 0.03)]], peaks)
     assert abs(tab2["qsub_kernel"]["us"] - 20.0) < 1e-9 and tab2["qsub_kernel"]["launches_per_step"] == 2
+
+
+def test_perq_tc_unions_counts_distinct_per_pair_tile():
+    sel = W.per_query_selection_large(2, 2, 64, 4000, 24, group=16, causal_prefix=3900)
+    u = bench.perq_tc_unions(sel, 8)
+    ref = [len(set(sel[g, t0:t0 + 16].flatten().tolist())) for g in range(2) for t0 in range(0, 64, 16)]
+    assert u == ref and len(u) == 8
