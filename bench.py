@@ -42,21 +42,20 @@ METRIC = "chunked-prefill sparse-attn tokens/s (select+attend) and % of roofline
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 def launches_per_step(w):
-    """Kernels one step launches.  Selection: query subselect (or, when every query is kept
-    and G * C <= 16, the decode shape, the kept queries' operand block for bf16 and nothing
-    for fp32), scoring and top-k.
+    """Kernels one step launches.  Selection: query subselect, scoring and top-k, or only
+    scoring and top-k when every query is kept and G * C <= 16 (the decode shape).
     Attention: the gather kernel and its combine when G * C <= 16, else compaction and
     the tensor-core kernel (bf16) or the CUDA-core kernel alone (fp32)."""
     small = w.group * w.chunk <= 16
-    sel = 3 if not (small and w.nq >= w.chunk) or w.dtype == "bf16" else 2
+    sel = 2 if small and w.nq >= w.chunk else 3
     att = 2 if small or w.dtype == "bf16" else 1
     return sel + att
 # DRAM traffic of one attention-kernel launch on the 128K-context workload
 # (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture of that kernel alone,
 # one launch, on this workload), valid only for the kernel sources it was taken on: the
 # digest below covers them, and a changed kernel reports null.
-ATTN_TRAFFIC = {"workload": "ctx_128k", "bytes": 117.494272e6 + 21.887744e6,
-                "sources": ['query_oriented_sparse_b200/csrc/attn_tc2.cuh', 'query_oriented_sparse_b200/csrc/tc_ptx.cuh'], "sha256_16": "e4300237fdf2f4d5"}
+ATTN_TRAFFIC = {"workload": "ctx_128k", "bytes": 117.528832e6 + 16.548608e6,
+                "sources": ['query_oriented_sparse_b200/csrc/attn_tc2.cuh', 'query_oriented_sparse_b200/csrc/tc_ptx.cuh'], "sha256_16": "d6ddd517e66da81a"}
 
 
 def attn_traffic(w):
@@ -96,8 +95,7 @@ def stage_model(w: W.Workload):
     return st
 
 
-KERNEL_STAGE = {"qsub_kernel": "qsub", "kept_all_prep_kernel": "qsub", "score_tc_kernel": "score",
-                "score_tc2_kernel": "score", "score_simt_kernel": "score",
+KERNEL_STAGE = {"qsub_kernel": "qsub", "score_tc_kernel": "score", "score_simt_kernel": "score",
                 "score_decode_kernel": "score", "topk_kernel": "topk", "topk_block_kernel": "topk",
                 "attn_tc2_kernel": "attn", "attn_tc_kernel": "attn", "attn_simt_kernel": "attn",
                 "attn_decode_kernel": "attn"}

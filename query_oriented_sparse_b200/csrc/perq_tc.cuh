@@ -61,14 +61,19 @@ perq_tc_union_kernel(const int32_t* __restrict__ sel, const __grid_constant__ Se
 
   for (int w = tid; w < W; w += PTC_THREADS) bm[w] = 0u;
   __syncthreads();
-  for (long long e = tid; e < 256LL * S; e += PTC_THREADS) {
-    const int rr = (int)(e / S), i = (int)(e - (long long)rr * S);
+  // a warp per row; a bit already set (most of them, when rows share their keys) costs a
+  // shared-memory read instead of an atomic
+  for (int rr = warp; rr < 256; rr += PTC_THREADS / 32) {
     int head, pos;
     if (!row_of(rr, head, pos)) continue;
-    const int x = sel[(((size_t)b * h_q + (size_t)g * G + head) * C + pos) * S + i];
-    if (x < 0) continue;
-    if (x >= N) { flag_error(ERR_BAD_INDEX); continue; }
-    atomicOr(&bm[x >> 5], 1u << (x & 31));
+    const int32_t* srow = sel + (((size_t)b * h_q + (size_t)g * G + head) * C + pos) * S;
+    for (int i = lane; i < S; i += 32) {
+      const int x = __ldg(srow + i);
+      if (x < 0) continue;
+      if (x >= N) { flag_error(ERR_BAD_INDEX); continue; }
+      const uint32_t bit = 1u << (x & 31);
+      if (!(bm[x >> 5] & bit)) atomicOr(&bm[x >> 5], bit);
+    }
   }
   __syncthreads();
   // exclusive scan of the words' popcounts (each thread a contiguous run of words)
@@ -128,7 +133,7 @@ perq_tc_union_kernel(const int32_t* __restrict__ sel, const __grid_constant__ Se
     if (row_of(rr, head, pos)) {
       const int32_t* srow = sel + (((size_t)b * h_q + (size_t)g * G + head) * C + pos) * S;
       for (int i = lane; i < S; i += 32) {
-        const int x = srow[i];
+        const int x = __ldg(srow + i);
         if (x < 0 || x >= N) continue;
         const uint32_t word = bm[x >> 5];
         const int rank = roff[x >> 5] + __popc(word & ((1u << (x & 31)) - 1u));
@@ -143,33 +148,33 @@ perq_tc_union_kernel(const int32_t* __restrict__ sel, const __grid_constant__ Se
 }
 
 // The union's K/V rows of every pair tile into blocks of `stride` rows (ascending union
-// order), zero rows up to the next multiple of 128.  Grid-stride over 16-byte vectors.
+// order), zero rows up to the next multiple of 128.  Grid (tiles, copiers per tile); each
+// CTA strides over its tile's 16-byte vectors.
 template <int VPR>
 __global__ void __launch_bounds__(256)
 perq_tc_gather_kernel(const uint4* __restrict__ k_cache, const uint4* __restrict__ v_cache,
                       long long rows_per_head, const __grid_constant__ SeqTable tab, int h_kv, int npt,
                       int cap, long long stride, const int32_t* __restrict__ uni,
-                      const int32_t* __restrict__ ucount, uint4* __restrict__ kc, uint4* __restrict__ vc,
-                      long long total_vecs) {
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total_vecs;
-       e += (long long)gridDim.x * blockDim.x) {
-    const long long rowg = e / VPR;
-    const int v = (int)(e - rowg * VPR);
-    const long long tile = rowg / stride;
-    const int i = (int)(rowg - tile * stride);
-    const int nu = __ldg(ucount + tile);
-    if (i >= (nu + 127) / 128 * 128) continue;               // never read
+                      const int32_t* __restrict__ ucount, uint4* __restrict__ kc, uint4* __restrict__ vc) {
+  const int tile = blockIdx.x;
+  const int nu = __ldg(ucount + tile);
+  const int nrow = (nu + 127) / 128 * 128;                     // rows the attention reads
+  const int bg = tile / npt;
+  const int b = bg / h_kv, g = bg - b * h_kv;
+  const long long src0 = (long long)g * rows_per_head + tab.kv_off[b];
+  const int32_t* U = uni + (size_t)tile * cap;
+  uint4* kt = kc + (size_t)tile * stride * VPR;
+  uint4* vt = vc + (size_t)tile * stride * VPR;
+  for (int e = blockIdx.y * blockDim.x + threadIdx.x; e < nrow * VPR; e += gridDim.y * blockDim.x) {
+    const int i = e / VPR, v = e - (e / VPR) * VPR;            // VPR is a power of two
     if (i >= nu) {
-      kc[e] = make_uint4(0u, 0u, 0u, 0u);
-      vc[e] = make_uint4(0u, 0u, 0u, 0u);
+      kt[e] = make_uint4(0u, 0u, 0u, 0u);
+      vt[e] = make_uint4(0u, 0u, 0u, 0u);
       continue;
     }
-    const int bg = (int)(tile / npt);
-    const int b = bg / h_kv, g = bg - b * h_kv;
-    const int x = __ldg(uni + tile * (size_t)cap + i);
-    const long long src = ((long long)g * rows_per_head + tab.kv_off[b] + x) * VPR + v;
-    kc[e] = __ldg(k_cache + src);
-    vc[e] = __ldg(v_cache + src);
+    const long long src = (src0 + __ldg(U + i)) * VPR + v;
+    kt[e] = __ldg(k_cache + src);
+    vt[e] = __ldg(v_cache + src);
   }
 }
 

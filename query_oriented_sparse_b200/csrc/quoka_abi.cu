@@ -14,7 +14,6 @@
 #include "qsub.cuh"
 #include "score_simt.cuh"
 #include "score_tc.cuh"
-#include "score_tc2.cuh"
 #include "topk.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
@@ -135,7 +134,6 @@ struct WsLayout {
   int ncg, heads_per_cg;    // column groups per KV head for the tensor-core scoring
   bool tc;                  // tensor-core scoring (bf16) or CUDA-core scoring (fp32)
   bool dec;                 // every query kept and <= 16 rows per KV head: decode scoring
-  bool dec_pair;            // decode shapes scored by the SM-pair tensor-core kernel (bf16)
 };
 
 WsLayout ws_layout(const Dims& d, int max_prefix, int nq) {
@@ -144,8 +142,7 @@ WsLayout ws_layout(const Dims& d, int max_prefix, int nq) {
   w.nkp = (w.nk + 15) / 16 * 16;
   w.dec = w.nk == d.C && d.G * d.C <= ADC_MAX_ROWS;
   w.tc = !w.dec && d.dt == QUOKA_BF16 && w.nkp <= STC_SLICE;
-  w.dec_pair = w.dec && d.dt == QUOKA_BF16 && ST2_SLICE % w.nkp == 0 && d.G * w.nkp <= ST2_MAXCOLS;
-  if (w.tc || w.dec_pair) {
+  if (w.tc) {
     // a column group is at most two head-aligned slices of <= 256 columns
     const int hmax = 2 * (STC_SLICE / w.nkp);
     w.ncg = (d.G + hmax - 1) / hmax;
@@ -287,50 +284,6 @@ quoka_status launch_score_tc(const Dims& d, const SeqTable& tab, long long rows,
   return QUOKA_OK;
 }
 
-// The SM-pair form of the scoring: 256-key pair tiles, slices of 128 columns (whole heads:
-// the kept queries per head, padded to 16, divide 128).  Decode shapes use it (WsLayout's
-// dec_pair).
-template <int D>
-quoka_status launch_score_tc2(const Dims& d, const SeqTable& tab, long long rows, const void* k,
-                              unsigned char* ws, const WsLayout& w, cudaStream_t st) {
-  ScoreTcParams p;
-  p.h_kv = d.h_kv;
-  p.G = d.G;
-  p.nkp = w.nkp;
-  p.ncg = w.ncg;
-  p.heads_per_cg = w.heads_per_cg;
-  p.padded = w.nk < w.nkp ? 1 : 0;
-  p.rows_per_head = rows;
-  p.pooled_stride = w.pooled_stride;
-  p.cg_stride = w.cg_stride;
-  p.inv_G = 1.0f / (float)d.G;
-  long long units = 0;
-  for (int b = 0; b < d.batch; ++b) {
-    p.unit_base[b] = (int)units;
-    units += (long long)d.h_kv * w.ncg * ((tab.prefix[b] + ST2_PT - 1) / ST2_PT);
-  }
-  for (int b = d.batch; b <= QUOKA_MAX_BATCH; ++b) p.unit_base[b] = (int)units;
-  if (units == 0) return QUOKA_OK;
-  if (units >= (1ll << 31)) return fail(QUOKA_ERR_UNSUPPORTED, "too many key tiles");
-  p.total_units = (int)units;
-  CUtensorMap kmap, qmap;
-  quoka_status s;
-  if ((s = make_map_bf16(&kmap, k, (uint64_t)d.h_kv * rows, D, 64, 128, "k_cache")) != QUOKA_OK) return s;
-  if ((s = make_map_bf16(&qmap, ws + w.qsel, (uint64_t)d.batch * d.h_q * w.nkp, D, 64, ST2_QBOX,
-                         "kept queries")) != QUOKA_OK)
-    return s;
-  cudaError_t e;
-  const int smem = St2Cfg<D>::SMEM;
-  if ((e = ensure_smem(score_tc2_kernel<D>, smem)) != cudaSuccess) return cuda_fail(e, "score_tc2 smem");
-  const int clusters = (int)std::min<long long>(units, sm_count() / 2);
-  score_tc2_kernel<D><<<2 * clusters, ST2_THREADS, smem, st>>>(
-      kmap, qmap, tab, p, reinterpret_cast<const float*>(ws + w.qinv),
-      reinterpret_cast<const float*>(ws + w.qbias), reinterpret_cast<float*>(ws + w.pooled));
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score_tc2 launch");
-  prof_mark(st, "score_tc2_kernel");
-  return QUOKA_OK;
-}
-
 // Top-B per (sequence, KV head): one CTA per row when there are many rows short enough to
 // stage in shared memory, else a 16-CTA cluster per row.
 quoka_status launch_topk(const Dims& d, const SeqTable& tab, int b_max, int32_t* idx_out,
@@ -409,19 +362,6 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
   float* pooled = reinterpret_cast<float*>(ws + w.pooled);
   cudaError_t e;
 
-  if (w.dec_pair) {
-    if constexpr (sizeof(T) == 2) {
-      kept_all_prep_kernel<T, D><<<d.batch * d.h_q, 128, 0, st>>>(
-          reinterpret_cast<const T*>(q), d.C, w.nkp, nq, qsel, qinv, qbias, kept_out);
-      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "kept_all_prep launch");
-      prof_mark(st, "kept_all_prep_kernel");
-      if (tab.max_prefix > 0) {
-        quoka_status s = launch_score_tc2<D>(d, tab, rows, k, ws, w, st);
-        if (s != QUOKA_OK) return s;
-      }
-      return launch_topk(d, tab, b_max, idx_out, w, pooled, st);
-    }
-  }
   if (w.dec) {
     quoka_status s = launch_select_decode<T, D>(d, tab, rows, q, k, nq, kept_out, pooled, w, st);
     if (s != QUOKA_OK) return s;
@@ -919,12 +859,11 @@ quoka_status launch_perq_tc(const Dims& d, const SeqTable& tab, long long rows, 
       sel, tab, d.h_q, d.h_kv, d.C, S, pl.TP, pl.cap, uni, ucount, mask);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_tc_union launch");
   prof_mark(st, "perq_tc_union_kernel");
-  const long long vecs = (long long)pl.tiles * pl.stride * 16;
-  const int grid = (int)std::min<long long>((vecs + 255) / 256, (long long)sm_count() * 16);
-  perq_tc_gather_kernel<16><<<grid, 256, 0, st>>>(
+  const int copiers = (int)std::max<long long>(1, std::min<long long>((pl.stride * 16 + 255) / 256,
+                                                                      (long long)sm_count() * 16 / pl.tiles + 1));
+  perq_tc_gather_kernel<16><<<dim3(pl.tiles, copiers), 256, 0, st>>>(
       reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), rows, tab, d.h_kv, pl.npt,
-      pl.cap, pl.stride, uni, ucount, reinterpret_cast<uint4*>(ws + pl.kc), reinterpret_cast<uint4*>(ws + pl.vc),
-      vecs);
+      pl.cap, pl.stride, uni, ucount, reinterpret_cast<uint4*>(ws + pl.kc), reinterpret_cast<uint4*>(ws + pl.vc));
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "perq_tc_gather launch");
   prof_mark(st, "perq_tc_gather_kernel");
   CUtensorMap qmap, kmap, vmap;

@@ -80,49 +80,6 @@ __device__ __forceinline__ void scd_vec16(const unsigned char* p, float (&x)[16 
   }
 }
 
-// Every query kept (decode shapes) and the scoring on tensor cores: the operand block of
-// the kept queries without a subselect.  One CTA per (sequence, query head): row t < C is
-// query t (raw), its 1/|q| (0 for a zero query) and bias 0; rows C .. nkp-1 are zero with
-// bias -inf, so they never win a max; kept_out (if asked) lists 0 .. C-1, then -1.
-template <typename T, int D>
-__global__ void __launch_bounds__(128)
-kept_all_prep_kernel(const T* __restrict__ q, int C, int nkp, int nq, T* __restrict__ qsel,
-                     float* __restrict__ qinv, float* __restrict__ qbias, int32_t* __restrict__ kept_out) {
-  constexpr int VPR = D * (int)sizeof(T) / 16;
-  const int bh = blockIdx.x;                   // b * h_q + h, row block bh * nkp
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int t = warp; t < nkp; t += 4) {
-    const size_t row = (size_t)bh * nkp + t;
-    uint4* dst = reinterpret_cast<uint4*>(qsel + row * D);
-    if (t < C) {
-      const uint4* src = reinterpret_cast<const uint4*>(q + ((size_t)bh * C + t) * D);
-      float ss = 0.f;
-      for (int v = lane; v < VPR; v += 32) {
-        const uint4 x = __ldg(src + v);
-        dst[v] = x;
-        float f[16 / sizeof(T)];
-        scd_vec16<T>(reinterpret_cast<const unsigned char*>(&x), f);
-#pragma unroll
-        for (int e = 0; e < (int)(16 / sizeof(T)); ++e) ss = fmaf(f[e], f[e], ss);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (lane == 0) {
-        qinv[row] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
-        qbias[row] = 0.f;
-      }
-    } else {
-      for (int v = lane; v < VPR; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
-      if (lane == 0) {
-        qinv[row] = 0.f;
-        qbias[row] = -INFINITY;
-      }
-    }
-  }
-  if (kept_out)
-    for (int i = threadIdx.x; i < nq; i += blockDim.x) kept_out[(size_t)bh * nq + i] = i < C ? i : -1;
-}
-
 // Rows r = j * C + t of a KV head: query head g*G + j, chunk position t (all kept).
 template <typename T, int D, int R>
 __global__ void __launch_bounds__(SCD_THREADS)

@@ -37,17 +37,17 @@ CASES = [
     # 3 heads of 112 padded rows per column group: two uneven head-aligned slices
     C("uneven_slices", h_q=12, h_kv=2, head_dim=128, chunk=150, prefix=3000, nq=100, budget=300,
       recipe="rank4", seed=17),
-    # SM-pair scoring: three 128-column slices per pair tile, the last pair tile past the
-    # prefix end on one CTA
-    C("pair_three_slices", h_q=6, h_kv=2, head_dim=128, chunk=300, prefix=2100, nq=128,
+    # three heads of 128 kept queries per KV head (accumulator slices of 256 and 128
+    # columns), a prefix that ends inside a key tile
+    C("g3_nq128", h_q=6, h_kv=2, head_dim=128, chunk=300, prefix=2100, nq=128,
       budget=300, recipe="heavy", seed=19),
-    # a 128-column and a 64-column slice, head_dim 64
-    C("pair_partial_slice_d64", h_q=3, h_kv=1, head_dim=64, chunk=100, prefix=700, nq=64,
+    # three heads of 64 kept queries, head_dim 64
+    C("g3_nq64_d64", h_q=3, h_kv=1, head_dim=64, chunk=100, prefix=700, nq=64,
       budget=96, seed=20),
-    # a 16-column slice: 8 query columns per SM of the pair
-    C("pair_n16", h_q=2, h_kv=2, head_dim=128, chunk=64, prefix=600, nq=16, budget=64, seed=21),
+    # one head of 16 kept queries per KV head: a 16-column accumulator slice
+    C("g1_nq16", h_q=2, h_kv=2, head_dim=128, chunk=64, prefix=600, nq=16, budget=64, seed=21),
     # two column groups of 8 heads per KV head, two sequences
-    C("pair_two_colgroups", h_q=16, h_kv=1, head_dim=128, chunk=128, prefix=(1500, 260), nq=64,
+    C("two_colgroups", h_q=16, h_kv=1, head_dim=128, chunk=128, prefix=(1500, 260), nq=64,
       budget=(200, 64), recipe="rank4", seed=22),
     # kept queries wider than one accumulator slice per head: CUDA-core scoring
     C("wide_nq", h_q=4, h_kv=2, head_dim=64, chunk=400, prefix=900, nq=300, budget=200, seed=18),
