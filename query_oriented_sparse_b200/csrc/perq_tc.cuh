@@ -24,6 +24,7 @@ namespace quoka {
 
 constexpr int PTC_THREADS = 1024;
 constexpr int PTC_MAX_WORDS = 8192;       // sequence bitmap: up to 262144 rows
+constexpr int PTC_BATCH = 8;              // set entries a lane has in flight
 
 // Shared memory of the union kernel: the sequence bitmap, its word offsets, and one
 // mask row per warp.
@@ -67,12 +68,20 @@ perq_tc_union_kernel(const int32_t* __restrict__ sel, const __grid_constant__ Se
     int head, pos;
     if (!row_of(rr, head, pos)) continue;
     const int32_t* srow = sel + (((size_t)b * h_q + (size_t)g * G + head) * C + pos) * S;
-    for (int i = lane; i < S; i += 32) {
-      const int x = __ldg(srow + i);
-      if (x < 0) continue;
-      if (x >= N) { flag_error(ERR_BAD_INDEX); continue; }
-      const uint32_t bit = 1u << (x & 31);
-      if (!(bm[x >> 5] & bit)) atomicOr(&bm[x >> 5], bit);
+    for (int i0 = 0; i0 < S; i0 += 32 * PTC_BATCH) {
+      int x[PTC_BATCH];                                        // all loads in flight first
+#pragma unroll
+      for (int u = 0; u < PTC_BATCH; ++u) {
+        const int i = i0 + u * 32 + lane;
+        x[u] = i < S ? __ldg(srow + i) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < PTC_BATCH; ++u) {
+        if (x[u] < 0) continue;
+        if (x[u] >= N) { flag_error(ERR_BAD_INDEX); continue; }
+        const uint32_t bit = 1u << (x[u] & 31);
+        if (!(bm[x[u] >> 5] & bit)) atomicOr(&bm[x[u] >> 5], bit);
+      }
     }
   }
   __syncthreads();
@@ -132,12 +141,20 @@ perq_tc_union_kernel(const int32_t* __restrict__ sel, const __grid_constant__ Se
     int head, pos;
     if (row_of(rr, head, pos)) {
       const int32_t* srow = sel + (((size_t)b * h_q + (size_t)g * G + head) * C + pos) * S;
-      for (int i = lane; i < S; i += 32) {
-        const int x = __ldg(srow + i);
-        if (x < 0 || x >= N) continue;
-        const uint32_t word = bm[x >> 5];
-        const int rank = roff[x >> 5] + __popc(word & ((1u << (x & 31)) - 1u));
-        if (rank < nu) atomicOr(&my[rank >> 5], 1u << (rank & 31));
+      for (int i0 = 0; i0 < S; i0 += 32 * PTC_BATCH) {
+        int x[PTC_BATCH];
+#pragma unroll
+        for (int u = 0; u < PTC_BATCH; ++u) {
+          const int i = i0 + u * 32 + lane;
+          x[u] = i < S ? __ldg(srow + i) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < PTC_BATCH; ++u) {
+          if (x[u] < 0 || x[u] >= N) continue;
+          const uint32_t word = bm[x[u] >> 5];
+          const int rank = roff[x[u] >> 5] + __popc(word & ((1u << (x[u] & 31)) - 1u));
+          if (rank < nu) atomicOr(&my[rank >> 5], 1u << (rank & 31));
+        }
       }
     }
     __syncwarp();
