@@ -24,6 +24,9 @@ CASES = [
     # one sequence, 16384 selected keys: 65 splits per KV head
     C("dec_bf16_128k", h_q=32, h_kv=8, head_dim=128, chunk=1, prefix=131072, nq=1,
       budget=16384, recipe="heavy", seed=32),
+    # 70000 selected keys for one KV head: hundreds of splits
+    C("dec_bf16_70k_splits", h_q=2, h_kv=1, head_dim=128, chunk=1, prefix=80000, nq=1,
+      budget=70000, recipe="heavy", seed=44),
     # G*C = 16 (R 16), d 64, a two-token chunk
     C("dec_bf16_d64_g8_c2", h_q=16, h_kv=2, head_dim=64, chunk=2, prefix=3000, nq=2, budget=400,
       recipe="rank4", seed=33),
