@@ -41,6 +41,7 @@ from query_oriented_sparse_b200 import workloads as W  # noqa: E402
 METRIC = "chunked-prefill sparse-attn tokens/s (select+attend) and % of roofline, 1 B200"
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024                       # B200 L2
 def launches_per_step(w):
     """Kernels one step launches.  Selection: query subselect, scoring and top-k, or only
     scoring and top-k when every query is kept and G * C <= 16 (the decode shape).
@@ -503,6 +504,11 @@ def run_ours(args, w):
         return run
 
     step_on = [make_step(0), make_step(1)]
+    # Between end-to-end steps the L2 is flushed inside the timed region unless the K/V
+    # cache the steps read is larger than twice the L2 by itself (then no step finds the
+    # previous one's keys in L2, and a flush would only add its own time).
+    kv_bytes = 2 * k.numel() * k.element_size()
+    e2e_flush = kv_bytes <= 2 * L2_BYTES
     for b in range(2):                     # fill both input buffers once, warm each call
         knb[b].copy_(kn_h)
         vnb[b].copy_(vn_h)
@@ -531,7 +537,8 @@ def run_ours(args, w):
             stream.wait_event(ev_in[b])
             if i >= 2:
                 stream.wait_event(ev_out[b])
-            flush.zero_()
+            if e2e_flush:
+                flush.zero_()
             step_on[b]()
             ev_cmp[b].record(stream)
             with torch.cuda.stream(s_out):
@@ -570,7 +577,9 @@ def run_ours(args, w):
                    "launch": launch_mode,
                    "parallelism": f"independent chunk step per GPU x{world}"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "l2": ("256 MB flush inside every end-to-end step" if e2e_flush else
+                       f"no flush: the K/V cache ({kv_bytes / 1e6:.0f} MB) is over twice the L2")},
         "gpu_launches": launches_per_step(w) * args.steps,
         "stage_us": {"select": statistics.mean(sel_ms) * 1e3,
                      "attn": statistics.mean(att_ms) * 1e3},
