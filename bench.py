@@ -97,7 +97,8 @@ def stage_model(w: W.Workload):
 
 
 KERNEL_STAGE = {"qsub_kernel": "qsub", "score_tc_kernel": "score", "score_simt_kernel": "score",
-                "score_decode_kernel": "score", "topk_kernel": "topk", "topk_block_kernel": "topk",
+                "score_decode_kernel": "score", "score_decode_tc_kernel": "score",
+                "topk_kernel": "topk", "topk_block_kernel": "topk",
                 "attn_tc2_kernel": "attn", "attn_tc_kernel": "attn", "attn_simt_kernel": "attn",
                 "attn_decode_kernel": "attn"}
 

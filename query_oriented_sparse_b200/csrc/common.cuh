@@ -38,6 +38,10 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
   return __float2bfloat16_rn(x);
 }
 
+// The two bf16 halves of a 32-bit word (low half = lower address) as floats.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
 // Load N consecutive elements (N * sizeof(T) is 8 or 16 bytes, aligned) as floats.
 template <typename T, int N>
 __device__ __forceinline__ void load_vec(const T* p, float (&out)[N]);

@@ -21,6 +21,7 @@
 #include "compact.cuh"
 #include "attn_decode.cuh"
 #include "select_decode.cuh"
+#include "score_decode_tc.cuh"
 #include "attn_perq.cuh"
 #include "selcache.cuh"
 #include "perq_tc.cuh"
@@ -326,8 +327,29 @@ quoka_status launch_score_decode_r(const Dims& d, const SeqTable& tab, long long
   return QUOKA_OK;
 }
 
+// bf16 decode scoring on tensor cores: a 128 x 16 MMA per 128-key tile, keys streamed
+// by TMA, two CTAs per SM.
+template <int D>
+quoka_status launch_score_decode_tc(const Dims& d, const SeqTable& tab, long long rows, const void* q,
+                                    const void* k, float* pooled, const WsLayout& w, cudaStream_t st) {
+  CUtensorMap kmap, qmap;
+  quoka_status s;
+  if ((s = make_map_bf16(&kmap, k, (uint64_t)d.h_kv * rows, D, 64, 128, "k_cache")) != QUOKA_OK) return s;
+  if ((s = make_map_bf16(&qmap, q, (uint64_t)d.batch * d.h_q * d.C, D, 64, SDT_QROWS, "q_chunk")) != QUOKA_OK)
+    return s;
+  cudaError_t e;
+  const int smem = SdtCfg<D>::SMEM;
+  if ((e = ensure_smem(score_decode_tc_kernel<D>, smem)) != cudaSuccess) return cuda_fail(e, "score_decode_tc smem");
+  dim3 grid((tab.max_prefix + SDT_TILES * 128 - 1) / (SDT_TILES * 128), d.h_kv, d.batch);
+  score_decode_tc_kernel<D><<<grid, SDT_THREADS, smem, st>>>(kmap, qmap, tab, rows, d.h_q, d.h_kv, d.C,
+                                                             pooled, w.pooled_stride);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "score_decode_tc launch");
+  prof_mark(st, "score_decode_tc_kernel");
+  return QUOKA_OK;
+}
+
 // Every query kept and at most 16 query rows per KV head: the kept positions are all of
-// them, and the scoring streams the prefix keys on CUDA cores.
+// them, and the scoring streams the prefix keys (bf16: tensor cores; fp32: CUDA cores).
 template <typename T, int D>
 quoka_status launch_select_decode(const Dims& d, const SeqTable& tab, long long rows, const void* q,
                                   const void* k, int nq, int32_t* kept_out, float* pooled,
@@ -341,6 +363,7 @@ quoka_status launch_select_decode(const Dims& d, const SeqTable& tab, long long 
     prof_mark(st, "kept_all_kernel");
   }
   if (tab.max_prefix == 0) return QUOKA_OK;
+  if constexpr (sizeof(T) == 2) return launch_score_decode_tc<D>(d, tab, rows, q, k, pooled, w, st);
   int r = 1;
   while (r < d.G * d.C) r *= 2;
   switch (r) {

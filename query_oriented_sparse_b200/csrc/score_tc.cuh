@@ -89,9 +89,6 @@ __device__ __forceinline__ void stc_next(const ScoreTcParams& p, const SeqTable&
   } while (tiles == 0);
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
 template <int D>
 __global__ void __launch_bounds__(STC_THREADS, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,

@@ -20,7 +20,7 @@ def test_kernel_timer_names_every_launch(kind, cuda_device):
     elif kind == "decode":
         w = W.custom("prof_decode", h_q=8, h_kv=2, head_dim=128, chunk=1, prefix=[3000] * 20,
                      nq=1, budget=384, recipe="heavy", seed=92)
-        expect = ["score_decode_kernel", "topk_block_kernel", "attn_decode_kernel",
+        expect = ["score_decode_tc_kernel", "topk_block_kernel", "attn_decode_kernel",
                   "attn_decode_combine_kernel"]
     else:
         w = W.custom("prof_f32", h_q=4, h_kv=1, head_dim=64, chunk=64, prefix=500, nq=8,
