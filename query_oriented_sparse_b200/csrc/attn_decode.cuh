@@ -24,7 +24,9 @@ namespace quoka {
 
 constexpr int ADC_MAX_ROWS = 16;      // query rows per KV head (G * C) this path takes
 constexpr int ADC_MIN_SPLIT = 256;    // keys per CTA at least (bounds the partials' bytes)
-constexpr int ADC_MAX_SPLIT = 4096;
+constexpr int ADC_MAX_SPLIT = 4096;   // unless that would need more than ADC_MAX_NSPLIT splits
+constexpr int ADC_MAX_NSPLIT = 512;   // splits per (sequence, KV head) at most
+constexpr int ADC_COMBINE_THREADS = 512;
 
 template <typename T, int D>
 struct AdcCfg {
@@ -294,38 +296,50 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 
 // Merges the splits of each (sequence b, KV head g): out = sum_s o_s 2^(m_s - M) /
 // sum_s l_s 2^(m_s - M), M the largest m_s.  Every row has at least its own chunk key,
-// so the denominator is positive.
+// so the denominator is positive.  The partials were just written and sit in L2, so the
+// merge is a few L2 round trips when its loads are in flight together: warp r reads row
+// r's (m, l) of every split at once (lane per split) and leaves each split's weight
+// 2^(m_s - M) in shared memory; then each thread takes output elements and loads that
+// element of up to eight splits before adding them in split order.
 template <typename T, int D, int R>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(ADC_COMBINE_THREADS)
 attn_decode_combine_kernel(const float* __restrict__ part, const __grid_constant__ SeqTable tab,
                            int h_q, int h_kv, int C, int split, int nsplit_ws, T* __restrict__ out) {
   constexpr int PD = D + 4;
-  __shared__ float Ms[R], Ls[R];
+  extern __shared__ float cw[];                            // [split][R] weights
+  __shared__ float Ls[R];
   const int g = blockIdx.x, b = blockIdx.y;
   const int G = h_q / h_kv, rows = G * C;
   const int nkeys = tab.nsel[b] + C;
   const int ns = (nkeys + split - 1) / split;
   const float* src = part + (size_t)(b * h_kv + g) * nsplit_ws * R * PD;
-  if (threadIdx.x < rows) {
-    const int r = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = warp; r < rows; r += ADC_COMBINE_THREADS / 32) {
     float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, src[((size_t)s * R + r) * PD + D]);
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, src[((size_t)s * R + r) * PD + D]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
-    for (int s = 0; s < ns; ++s) {
+    for (int s = lane; s < ns; s += 32) {
       const float ms = src[((size_t)s * R + r) * PD + D];
-      if (ms != -INFINITY) L += src[((size_t)s * R + r) * PD + D + 1] * exp2f(ms - M);
+      const float e = ms != -INFINITY ? exp2f(ms - M) : 0.f;   // an empty split weighs 0
+      cw[s * R + r] = e;
+      if (ms != -INFINITY) L += src[((size_t)s * R + r) * PD + D + 1] * e;
     }
-    Ms[r] = M;
-    Ls[r] = L;
+    L = warp_sum(L);
+    if (lane == 0) Ls[r] = L;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < rows * D; e += blockDim.x) {
+  for (int e = threadIdx.x; e < rows * D; e += ADC_COMBINE_THREADS) {
     const int r = e / D, d = e - r * D;
-    const float M = Ms[r];
     float o = 0.f;
-    for (int s = 0; s < ns; ++s) {
-      const float ms = src[((size_t)s * R + r) * PD + D];
-      if (ms != -INFINITY) o += src[((size_t)s * R + r) * PD + d] * exp2f(ms - M);
+    for (int s0 = 0; s0 < ns; s0 += 8) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = s0 + u < ns ? src[((size_t)(s0 + u) * R + r) * PD + d] : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (s0 + u < ns) o = fmaf(x[u], cw[(s0 + u) * R + r], o);
     }
     const int j = r / C, t = r - j * C;
     out[(((size_t)b * h_q + (size_t)g * G + j) * C + t) * D + d] = from_f32<T>(o / Ls[r]);

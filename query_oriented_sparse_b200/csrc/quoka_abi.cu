@@ -554,6 +554,10 @@ quoka_status launch_attn_decode_r(const Dims& d, const SeqTable& tab, long long 
   long long split = (total + target - 1) / target;
   split = (split + 32 * Cfg::NW - 1) / (32 * Cfg::NW) * (32 * Cfg::NW);
   split = std::min<long long>(std::max<long long>(split, ADC_MIN_SPLIT), ADC_MAX_SPLIT);
+  if ((nmax + split - 1) / split > ADC_MAX_NSPLIT) {        // the merge stages one weight per split
+    split = (nmax + ADC_MAX_NSPLIT - 1) / ADC_MAX_NSPLIT;
+    split = (split + 32 * Cfg::NW - 1) / (32 * Cfg::NW) * (32 * Cfg::NW);
+  }
   const int nsplit = (int)((nmax + split - 1) / split);
   const int nsplit_ws = decode_nsplit_ws(d, b_max);
   const int smem = adc_smem_bytes<T, D, R>();
@@ -566,7 +570,7 @@ quoka_status launch_attn_decode_r(const Dims& d, const SeqTable& tab, long long 
       rows, tab, d.h_q, d.h_kv, d.C, idx, idx_stride, (int)split, nsplit_ws, scale_log2, part);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode launch");
   prof_mark(st, "attn_decode_kernel");
-  attn_decode_combine_kernel<T, D, R><<<dim3(d.h_kv, d.batch), 128, 0, st>>>(
+  attn_decode_combine_kernel<T, D, R><<<dim3(d.h_kv, d.batch), ADC_COMBINE_THREADS, nsplit * R * 4, st>>>(
       part, tab, d.h_q, d.h_kv, d.C, (int)split, nsplit_ws, reinterpret_cast<T*>(out));
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode combine launch");
   prof_mark(st, "attn_decode_combine_kernel");
