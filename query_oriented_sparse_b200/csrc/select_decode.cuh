@@ -20,6 +20,7 @@
 #pragma once
 #include "cluster_select.cuh"
 #include "tc_ptx.cuh"
+#include "topk.cuh"
 
 namespace quoka {
 
@@ -227,14 +228,27 @@ topk_block_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, 
     return;
   }
   if (B == 0) return;
-  for (int j = threadIdx.x; j < P; j += blockDim.x) {
-    float s = sc[j];
-    if (ncg > 1) {                                         // column groups, in group order
-      for (int c = 1; c < ncg; ++c) s += sc[c * cg_stride + j];
-      s *= inv_G;
-      sc[j] = s;
+  // stage the row's keys: TOPK_STAGE_UNROLL loads in flight per thread (the scores were
+  // just written and sit in L2, so the staging costs a few round trips, not one per key)
+  for (int j0 = threadIdx.x; j0 < P; j0 += TOPK_STAGE_UNROLL * blockDim.x) {
+    float v[TOPK_STAGE_UNROLL];
+#pragma unroll
+    for (int u = 0; u < TOPK_STAGE_UNROLL; ++u) {
+      const int j = j0 + u * blockDim.x;
+      v[u] = j < P ? sc[j] : 0.f;
     }
-    staged[j] = float_to_ordered(s);
+#pragma unroll
+    for (int u = 0; u < TOPK_STAGE_UNROLL; ++u) {
+      const int j = j0 + u * blockDim.x;
+      if (j >= P) continue;
+      float s = v[u];
+      if (ncg > 1) {                                       // column groups, in group order
+        for (int c = 1; c < ncg; ++c) s += sc[c * cg_stride + j];
+        s *= inv_G;
+        sc[j] = s;
+      }
+      staged[j] = float_to_ordered(s);
+    }
   }
   __syncthreads();
   auto key_at = [&](int j) { return staged[j]; };
