@@ -100,7 +100,8 @@ quoka_status quoka_workspace_pooled_view(const quoka_shape* shape, int max_prefi
  * the attention call always adds them causally, so budget[b] counts prefix keys.
  * When every query is kept (nq >= chunk) and at most 16 query rows share a KV head (a
  * decode step, C = 1, or a short chunk), steps 1-2 are trivial and step 3 runs as a
- * stream over the keys on CUDA cores; the result is the same.
+ * stream over the keys (bf16: a 128 x 16 tensor-core MMA per 128-key tile; fp32: CUDA
+ * cores); the result is the same.
  *
  *   q_chunk     device, [batch, h_q, chunk, head_dim]
  *   k_cache     device, [h_kv, kv_off[batch], head_dim]

@@ -3,9 +3,9 @@
 // and at most 16 query rows share a KV head.
 //
 // With one or a few kept queries per head the cosine scoring is a stream over the prefix
-// keys with a handful of dot products per key, bound by reading the keys: a 128-key
-// tensor-core tile would carry a few useful columns and pay a fixed hand-off latency per
-// tile.  So:
+// keys with a handful of dot products per key, bound by reading the keys.  bf16 keys are
+// scored by score_decode_tc_kernel (score_decode_tc.cuh: TMA-streamed tiles, a 128 x 16
+// tensor-core MMA per tile); fp32 keys here:
 //   kept_all_kernel      writes the kept positions (all of them) when the caller asks;
 //   score_decode_kernel  one CTA per (1024-key tile, KV head, sequence), four warps; each
 //                        warp streams batches of 32 consecutive key rows into its own
