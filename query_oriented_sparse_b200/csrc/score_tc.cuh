@@ -335,44 +335,64 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         for (int kb = 0; kb < KB; ++kb) ptx::mbar_arrive(&kempty[st[kb]]);
       if (!ok) break;
 
-      // sum over this group's heads of max over the head's kept queries of s / |q| (+ bias)
+      // sum over this group's heads of max over the head's kept queries of s / |q| (+ bias):
+      // whole 32-column chunks (one tcgen05.ld each) in straight-line code, then a 16-column
+      // tail when the head's width is an odd multiple of 16
       auto range_max = [&](uint32_t tcol, int cbase, int ncol) -> float {
         const float* ci = cpi + cbase;
         const float* cb = cpb + cbase;
         float run = -INFINITY;
-        for (int c = 0; c < ncol; c += 32) {
-          const int w = min(32, ncol - c);         // 32 or (odd tail) 16 columns
+        int c = 0;
+        for (; c + 32 <= ncol; c += 32) {
           uint32_t r[32];
-          if (w == 32) ptx::tmem_ld32(lane_base + tcol + (uint32_t)c, r);
-          else ptx::tmem_ld16(lane_base + tcol + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(r));
+          ptx::tmem_ld32(lane_base + tcol + (uint32_t)c, r);
           ptx::tmem_ld_wait();
+          float v[32];
+          if (p.padded) {
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            if (q * 16 < w) {
-              float v[16];
+            for (int i = 0; i < 32; i += 4) {
+              const float4 sc = *reinterpret_cast<const float4*>(ci + c + i);
+              const float4 bi = *reinterpret_cast<const float4*>(cb + c + i);
+              v[i] = fmaf(__uint_as_float(r[i]), sc.x, bi.x);
+              v[i + 1] = fmaf(__uint_as_float(r[i + 1]), sc.y, bi.y);
+              v[i + 2] = fmaf(__uint_as_float(r[i + 2]), sc.z, bi.z);
+              v[i + 3] = fmaf(__uint_as_float(r[i + 3]), sc.w, bi.w);
+            }
+          } else {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float4 sc = reinterpret_cast<const float4*>(ci + c + q * 16)[i];
-                const uint32_t* rr = &r[q * 16 + 4 * i];
-                const float2 s01 = make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1]));
-                const float2 s23 = make_float2(__uint_as_float(rr[2]), __uint_as_float(rr[3]));
-                float2 v01, v23;
-                if (p.padded) {
-                  const float4 bi = reinterpret_cast<const float4*>(cb + c + q * 16)[i];
-                  v01 = ptx::fma2(s01, make_float2(sc.x, sc.y), make_float2(bi.x, bi.y));
-                  v23 = ptx::fma2(s23, make_float2(sc.z, sc.w), make_float2(bi.z, bi.w));
-                } else {
-                  v01 = ptx::mul2(s01, make_float2(sc.x, sc.y));
-                  v23 = ptx::mul2(s23, make_float2(sc.z, sc.w));
-                }
-                v[4 * i] = v01.x; v[4 * i + 1] = v01.y; v[4 * i + 2] = v23.x; v[4 * i + 3] = v23.y;
-              }
-              const float a0 = ptx::max3(v[0], v[1], v[2]), a1 = ptx::max3(v[3], v[4], v[5]);
-              const float a2 = ptx::max3(v[6], v[7], v[8]), a3 = ptx::max3(v[9], v[10], v[11]);
-              const float a4 = ptx::max3(v[12], v[13], v[14]);
-              run = ptx::max3(run, ptx::max3(a0, a1, a2), ptx::max3(a3, a4, v[15]));
+            for (int i = 0; i < 32; i += 4) {
+              const float4 sc = *reinterpret_cast<const float4*>(ci + c + i);
+              const float2 v01 = ptx::mul2(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), make_float2(sc.x, sc.y));
+              const float2 v23 = ptx::mul2(make_float2(__uint_as_float(r[i + 2]), __uint_as_float(r[i + 3])), make_float2(sc.z, sc.w));
+              v[i] = v01.x; v[i + 1] = v01.y; v[i + 2] = v23.x; v[i + 3] = v23.y;
             }
           }
+          float a[11];
+#pragma unroll
+          for (int k = 0; k < 10; ++k) a[k] = ptx::max3(v[3 * k], v[3 * k + 1], v[3 * k + 2]);
+          a[10] = fmaxf(v[30], v[31]);
+          const float b0 = ptx::max3(a[0], a[1], a[2]), b1 = ptx::max3(a[3], a[4], a[5]);
+          const float b2 = ptx::max3(a[6], a[7], a[8]), b3 = fmaxf(a[9], a[10]);
+          run = ptx::max3(run, ptx::max3(b0, b1, b2), b3);
+        }
+        if (c < ncol) {                              // 16-column tail
+          uint32_t r[16];
+          ptx::tmem_ld16(lane_base + tcol + (uint32_t)c, r);
+          ptx::tmem_ld_wait();
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float4 sc = *reinterpret_cast<const float4*>(ci + c + i);
+            const float4 bi = p.padded ? *reinterpret_cast<const float4*>(cb + c + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[i] = fmaf(__uint_as_float(r[i]), sc.x, bi.x);
+            v[i + 1] = fmaf(__uint_as_float(r[i + 1]), sc.y, bi.y);
+            v[i + 2] = fmaf(__uint_as_float(r[i + 2]), sc.z, bi.z);
+            v[i + 3] = fmaf(__uint_as_float(r[i + 3]), sc.w, bi.w);
+          }
+          const float a0 = ptx::max3(v[0], v[1], v[2]), a1 = ptx::max3(v[3], v[4], v[5]);
+          const float a2 = ptx::max3(v[6], v[7], v[8]), a3 = ptx::max3(v[9], v[10], v[11]);
+          const float a4 = ptx::max3(v[12], v[13], v[14]);
+          run = ptx::max3(run, ptx::max3(a0, a1, a2), ptx::max3(a3, a4, v[15]));
         }
         return run;
       };
