@@ -226,7 +226,24 @@ qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
     for (int t = lo + tid; t < hi; t += blockDim.x) emit(t, t);
   } else {
     cluster.sync();                            // every CTA's keys are final
-    {                                          // all remote loads in flight before any store
+    // all remote loads in flight before any store; 16-byte pulls when every CTA's slice
+    // starts on a 16-byte boundary (C a multiple of 32), else 4-byte ones
+    if ((S & 3) == 0 && (C & 3) == 0) {
+      constexpr int PULL4 = (QSUB_PULL + 3) / 4;
+      uint4 v[PULL4];
+#pragma unroll
+      for (int i = 0; i < PULL4; ++i) {
+        const int t = (tid + i * QSUB_THREADS) * 4;
+        v[i] = (t < C && t / S != rank)
+                   ? *reinterpret_cast<const uint4*>(cluster.map_shared_rank(keys, t / S) + t)
+                   : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < PULL4; ++i) {
+        const int t = (tid + i * QSUB_THREADS) * 4;
+        if (t < C && t / S != rank) *reinterpret_cast<uint4*>(keys + t) = v[i];
+      }
+    } else {
       uint32_t v[QSUB_PULL];
 #pragma unroll
       for (int i = 0; i < QSUB_PULL; ++i) {
