@@ -212,7 +212,12 @@ score_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       }
       const float nn = nn2.x + nn2.y;
       const int j = j0 + t * 128 + row;
-      if (j < P) out[j] = nn > 0.f ? (s * inv_G) / sqrtf(nn) : 0.f;
+      if (j < P) {
+        const float val = nn > 0.f ? (s * inv_G) / sqrtf(nn) : 0.f;
+        uint64_t pol;
+        asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+        asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(out + j), "f"(val), "l"(pol) : "memory");
+      }
     }
   }
 
