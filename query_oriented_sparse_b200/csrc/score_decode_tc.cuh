@@ -12,7 +12,9 @@
 // and write
 //     s = (1/G) sum_h max_t (q_{h,t} . k / |q_{h,t}|) / |k|.
 // 1/|q| of each row is taken once per CTA from the query block in shared memory, so
-// the only HBM traffic is one read of the keys and the pooled-score write.
+// the only HBM traffic is one read of the keys and the pooled-score write.  The pooled
+// scores are stored with an L2 evict-last policy, so the key stream behind them does not
+// push them out before the top-k reads them.
 //
 // One CTA per (span of SDT_TILES tiles, KV head, sequence); two CTAs fit on an SM, so one
 // streams while the other starts or drains.  Warp 0 loads, warp 1 issues the MMAs,
@@ -212,7 +214,7 @@ score_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       }
       const float nn = nn2.x + nn2.y;
       const int j = j0 + t * 128 + row;
-      if (j < P) {
+      if (j < P) {                                         // the top-k reads it next: keep it in L2
         const float val = nn > 0.f ? (s * inv_G) / sqrtf(nn) : 0.f;
         uint64_t pol;
         asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
