@@ -363,15 +363,18 @@ quoka_status launch_select_decode(const Dims& d, const SeqTable& tab, long long 
     prof_mark(st, "kept_all_kernel");
   }
   if (tab.max_prefix == 0) return QUOKA_OK;
-  if constexpr (sizeof(T) == 2) return launch_score_decode_tc<D>(d, tab, rows, q, k, pooled, w, st);
-  int r = 1;
-  while (r < d.G * d.C) r *= 2;
-  switch (r) {
-    case 1: return launch_score_decode_r<T, D, 1>(d, tab, rows, q, k, pooled, w, st);
-    case 2: return launch_score_decode_r<T, D, 2>(d, tab, rows, q, k, pooled, w, st);
-    case 4: return launch_score_decode_r<T, D, 4>(d, tab, rows, q, k, pooled, w, st);
-    case 8: return launch_score_decode_r<T, D, 8>(d, tab, rows, q, k, pooled, w, st);
-    default: return launch_score_decode_r<T, D, 16>(d, tab, rows, q, k, pooled, w, st);
+  if constexpr (sizeof(T) == 2) {
+    return launch_score_decode_tc<D>(d, tab, rows, q, k, pooled, w, st);
+  } else {
+    int r = 1;
+    while (r < d.G * d.C) r *= 2;
+    switch (r) {
+      case 1: return launch_score_decode_r<T, D, 1>(d, tab, rows, q, k, pooled, w, st);
+      case 2: return launch_score_decode_r<T, D, 2>(d, tab, rows, q, k, pooled, w, st);
+      case 4: return launch_score_decode_r<T, D, 4>(d, tab, rows, q, k, pooled, w, st);
+      case 8: return launch_score_decode_r<T, D, 8>(d, tab, rows, q, k, pooled, w, st);
+      default: return launch_score_decode_r<T, D, 16>(d, tab, rows, q, k, pooled, w, st);
+    }
   }
 }
 

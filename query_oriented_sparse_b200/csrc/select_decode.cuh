@@ -150,49 +150,24 @@ score_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, long long 
     const unsigned char* krow = stage + (bt & 1) * Cfg::STAGE + lane * ROW;
     float dot[R];
     float nn = 0.f;
-    if constexpr (sizeof(T) == 2) {
-      // bf16 keys: even and odd dimensions in the two halves of packed fp32x2 FMAs
-      float2 dot2[R], nn2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int r = 0; r < R; ++r) dot2[r] = make_float2(0.f, 0.f);
+    for (int r = 0; r < R; ++r) dot[r] = 0.f;
 #pragma unroll 2
-      for (int c = 0; c < VPR; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(krow + c * 16);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int c = 0; c < VPR; ++c) {
+      float kx[EPV];
+      scd_vec16<T>(krow + c * 16, kx);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 k2 = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-          nn2 = ptx::fma2(k2, k2, nn2);
+      for (int e = 0; e < EPV; ++e) nn = fmaf(kx[e], kx[e], nn);
 #pragma unroll
-          for (int r = 0; r < R; ++r) {
-            const float2 q2 = *reinterpret_cast<const float2*>(qs + r * D + c * EPV + 2 * i);
-            dot2[r] = ptx::fma2(q2, k2, dot2[r]);
-          }
-        }
-      }
+      for (int r = 0; r < R; ++r) {
+        const float* qr = qs + r * D + c * EPV;
 #pragma unroll
-      for (int r = 0; r < R; ++r) dot[r] = dot2[r].x + dot2[r].y;
-      nn = nn2.x + nn2.y;
-    } else {
-#pragma unroll
-      for (int r = 0; r < R; ++r) dot[r] = 0.f;
-#pragma unroll 2
-      for (int c = 0; c < VPR; ++c) {
-        float kx[EPV];
-        scd_vec16<T>(krow + c * 16, kx);
-#pragma unroll
-        for (int e = 0; e < EPV; ++e) nn = fmaf(kx[e], kx[e], nn);
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const float* qr = qs + r * D + c * EPV;
-#pragma unroll
-          for (int e4 = 0; e4 < EPV; e4 += 4) {
-            const float4 qv = *reinterpret_cast<const float4*>(qr + e4);
-            dot[r] = fmaf(qv.x, kx[e4], dot[r]);
-            dot[r] = fmaf(qv.y, kx[e4 + 1], dot[r]);
-            dot[r] = fmaf(qv.z, kx[e4 + 2], dot[r]);
-            dot[r] = fmaf(qv.w, kx[e4 + 3], dot[r]);
-          }
+        for (int e4 = 0; e4 < EPV; e4 += 4) {
+          const float4 qv = *reinterpret_cast<const float4*>(qr + e4);
+          dot[r] = fmaf(qv.x, kx[e4], dot[r]);
+          dot[r] = fmaf(qv.y, kx[e4 + 1], dot[r]);
+          dot[r] = fmaf(qv.z, kx[e4 + 2], dot[r]);
+          dot[r] = fmaf(qv.w, kx[e4 + 3], dot[r]);
         }
       }
     }
