@@ -66,6 +66,7 @@ struct Attn2Params {
   int h_q, h_kv, G, C, TP;
   long long kc_stride;             // rows per (sequence, KV head) block of the compacted cache
   float scale_log2;                // log2(e) / sqrt(d)
+  int border[QUOKA_MAX_BATCH];     // grid z -> sequence, longest key lists first
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -109,7 +110,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster.block_rank();
-  const int b = blockIdx.z, g = blockIdx.y;
+  const int b = p.border[blockIdx.z], g = blockIdx.y;
   const int npairs = (p.C + 2 * p.TP - 1) / (2 * p.TP);
   const int pair = npairs - 1 - (int)(blockIdx.x >> 1);     // longest key ranges first
   const int t0 = pair * 2 * p.TP;

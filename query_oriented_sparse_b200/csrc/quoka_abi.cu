@@ -485,6 +485,15 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
   return launch_attn_tc_core<D>(d, tab, q, kc, vc, p.kc_stride, out, st);
 }
 
+// Grid z -> sequence for the pair attention: sequences with the most keys first, so a
+// ragged batch's longest pairs start early and the last wave holds the shortest ones.
+void fill_border(Attn2Params& p2, const Dims& d, const SeqTable& tab) {
+  std::vector<int> order(d.batch);
+  for (int b = 0; b < d.batch; ++b) order[b] = b;
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return tab.nsel[x] > tab.nsel[y]; });
+  for (int i = 0; i < QUOKA_MAX_BATCH; ++i) p2.border[i] = i < d.batch ? order[i] : 0;
+}
+
 // The tensor-core attention over compacted blocks kc / vc of kc_stride rows per
 // (sequence, KV head): selected rows first, then the chunk rows, then zero rows.
 template <int D>
@@ -517,6 +526,7 @@ quoka_status launch_attn_tc_core(const Dims& d, const SeqTable& tab, const void*
     p2.TP = p.TP;
     p2.kc_stride = p.kc_stride;
     p2.scale_log2 = p.scale_log2;
+    fill_border(p2, d, tab);
     const int smem2 = At2Cfg::SMEM;
     if ((e = ensure_smem(attn_tc2_kernel<false>, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
     dim3 grid2(2 * ((d.C + 2 * p.TP - 1) / (2 * p.TP)), d.h_kv, d.batch);
@@ -910,6 +920,7 @@ quoka_status launch_perq_tc(const Dims& d, const SeqTable& tab, long long rows, 
   p2.TP = pl.TP;
   p2.kc_stride = pl.stride;
   p2.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
+  for (int i = 0; i < QUOKA_MAX_BATCH; ++i) p2.border[i] = i;   // unions are sized on the device
   const int smem2 = At2Cfg::SMEM;
   if ((e = ensure_smem(attn_tc2_kernel<true>, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
   attn_tc2_kernel<true><<<dim3(2 * pl.npt, d.h_kv, d.batch), AT2_THREADS, smem2, st>>>(
