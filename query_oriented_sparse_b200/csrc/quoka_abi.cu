@@ -487,6 +487,33 @@ quoka_status launch_attn_tc(const Dims& d, const SeqTable& tab, long long rows, 
 
 // Grid z -> sequence for the pair attention: sequences with the most keys first, so a
 // ragged batch's longest pairs start early and the last wave holds the shortest ones.
+// Clusters (SM pairs) of the pair attention kernel that fit on the device at once: the
+// persistent grid's size.  Queried once per (device, kernel form).
+#ifndef AT2_PERSIST_MAX_BLOCKS
+#define AT2_PERSIST_MAX_BLOCKS 100   // mean 128-key blocks per tile up to which the grid is persistent
+#endif
+template <bool kMember, bool kPersist>
+int at2_resident_pairs(int smem) {
+  static std::mutex mu;
+  static std::map<int, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * sm_count(), 1, 1);
+  cfg.blockDim = dim3(AT2_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (const void*)attn_tc2_kernel<kMember, kPersist>, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    n = sm_count() / 2;
+  }
+  cache[dev] = n;
+  return n;
+}
+
 void fill_border(Attn2Params& p2, const Dims& d, const SeqTable& tab) {
   std::vector<int> order(d.batch);
   for (int b = 0; b < d.batch; ++b) order[b] = b;
@@ -527,12 +554,27 @@ quoka_status launch_attn_tc_core(const Dims& d, const SeqTable& tab, const void*
     p2.kc_stride = p.kc_stride;
     p2.scale_log2 = p.scale_log2;
     fill_border(p2, d, tab);
-    const int smem2 = At2Cfg::SMEM;
-    if ((e = ensure_smem(attn_tc2_kernel<false>, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
-    dim3 grid2(2 * ((d.C + 2 * p.TP - 1) / (2 * p.TP)), d.h_kv, d.batch);
-    attn_tc2_kernel<false><<<grid2, AT2_THREADS, smem2, st>>>(qmap, kmap, vmap, tab, p2,
-                                                              reinterpret_cast<__nv_bfloat16*>(out),
-                                                              nullptr, nullptr, 0);
+    // One cluster per tile, or, when there are more tiles than resident clusters and the
+    // tiles are short (their fill and drain then weigh more than what the hardware's
+    // dynamic order of whole tiles gains), as many clusters as fit, each walking the list.
+    const int npairs2 = (d.C + 2 * p.TP - 1) / (2 * p.TP);
+    const long long tiles = (long long)npairs2 * d.h_kv * d.batch;
+    long long blocks = 0;
+    for (int b = 0; b < d.batch; ++b)
+      for (int pr = 0; pr < npairs2; ++pr)
+        blocks += (long long)d.h_kv * ((tab.nsel[b] + std::min(d.C, (pr + 1) * 2 * p.TP) + 127) / 128);
+    const int smem_p = At2Cfg::smem(true);
+    if ((e = ensure_smem(attn_tc2_kernel<false, true>, smem_p)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
+    const long long ncl = at2_resident_pairs<false, true>(smem_p);
+    if (tiles > ncl && blocks <= (long long)AT2_PERSIST_MAX_BLOCKS * tiles) {
+      attn_tc2_kernel<false, true><<<dim3(2 * (unsigned)ncl), AT2_THREADS, smem_p, st>>>(
+          qmap, kmap, vmap, tab, p2, reinterpret_cast<__nv_bfloat16*>(out), nullptr, nullptr, 0);
+    } else {
+      const int smem2 = At2Cfg::smem(false);
+      if ((e = ensure_smem(attn_tc2_kernel<false, false>, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
+      attn_tc2_kernel<false, false><<<dim3(2 * npairs2, d.h_kv, d.batch), AT2_THREADS, smem2, st>>>(
+          qmap, kmap, vmap, tab, p2, reinterpret_cast<__nv_bfloat16*>(out), nullptr, nullptr, 0);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_tc2 launch");
     prof_mark(st, "attn_tc2_kernel");
     return QUOKA_OK;
@@ -921,9 +963,9 @@ quoka_status launch_perq_tc(const Dims& d, const SeqTable& tab, long long rows, 
   p2.kc_stride = pl.stride;
   p2.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
   for (int i = 0; i < QUOKA_MAX_BATCH; ++i) p2.border[i] = i;   // unions are sized on the device
-  const int smem2 = At2Cfg::SMEM;
-  if ((e = ensure_smem(attn_tc2_kernel<true>, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
-  attn_tc2_kernel<true><<<dim3(2 * pl.npt, d.h_kv, d.batch), AT2_THREADS, smem2, st>>>(
+  const int smem2 = At2Cfg::smem(false);
+  if ((e = ensure_smem(attn_tc2_kernel<true, false>, smem2)) != cudaSuccess) return cuda_fail(e, "attn_tc2 smem");
+  attn_tc2_kernel<true, false><<<dim3(2 * pl.npt, d.h_kv, d.batch), AT2_THREADS, smem2, st>>>(
       qmap, kmap, vmap, tab, p2, reinterpret_cast<__nv_bfloat16*>(out), mask, ucount, pl.mwords);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_tc2 (per-query) launch");
   prof_mark(st, "attn_tc2_kernel");
