@@ -8,13 +8,14 @@
 // place of the causal rule (perq_tc.cuh builds the union, the masks and the K/V block).
 //
 // A cluster of two CTAs on two SMs serves (sequence, KV head, 2 x TP chunk positions)
-// tiles in turn: the grid holds as many clusters as can be resident at once, and cluster c
-// takes tiles c, c + N, c + 2N, ... of the list ordered by sequence (most selected keys
-// first), KV head and pair (longest key range first), keeping its TMEM, barriers and
-// pipeline across tiles, so the next tile's query gather, K/V loads and first S MMAs run
-// while the current tile drains.  CTA r owns query tile r: 128 rows packing the G query
-// heads of the KV head at TP = 128 / G positions, gathered by TMA (tile::gather4) into one
-// of two query buffers.  The pair runs every
+// tiles, listed by sequence (most selected keys first), KV head and pair (longest key
+// range first).  Either one cluster per tile (kPersist = false), or (kPersist = true) the
+// grid holds as many clusters as can be resident at once and cluster c takes tiles c,
+// c + N, c + 2N, ... of the list, keeping its TMEM, barriers and pipeline across tiles, so
+// the next tile's query gather (into a second query buffer), K/V loads and first S MMAs
+// run while the current tile drains.  CTA r owns query tile r: 128 rows packing the G
+// query heads of the KV head at TP = 128 / G positions, gathered by TMA (tile::gather4).
+// The pair runs every
 // MMA as one 256-row tcgen05.mma (cta_group::2) issued by one thread of CTA 0:
 //   S = Q K^T   (M 256, N 128 keys, K d): A = each CTA's query tile, B = the 128-key
 //               tile split by keys, CTA r holding keys 64r .. 64r+63;
