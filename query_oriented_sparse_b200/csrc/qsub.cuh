@@ -2,8 +2,11 @@
 // queries are filtered by cosine dissimilarity to their mean; Figure 2: queries far
 // from the mean interact with more keys).
 //
-// One thread-block cluster of QSUB_CS CTAs per (sequence, query head); CTA r owns a
-// contiguous slice of the chunk positions.  Rows are read eight lanes to a row (a warp
+// One thread-block cluster of CS CTAs per (sequence, query head); CTA r owns a contiguous
+// slice of at most QSUB_MAX_ROWS chunk positions.  The call takes the smallest CS that
+// covers the chunk and doubles it while the clusters of all heads still fit the SMs at
+// once, so a long chunk of few heads spreads over 8 SMs and many short heads each run on
+// one (the select's latency chain then runs once per SM, not once per wave of clusters).  Rows are read eight lanes to a row (a warp
 // takes four rows per step, each lane one or more 16-byte vectors), several steps in
 // flight per warp, so a row's reductions are three shuffles wide instead of a serial
 // five-shuffle chain per row.
@@ -25,10 +28,10 @@
 
 namespace quoka {
 
-constexpr int QSUB_CS = 8;                    // CTAs per query head
+constexpr int QSUB_MAX_CS = 8;                // CTAs per query head at most
 constexpr int QSUB_THREADS = 512;
 constexpr int QSUB_WARPS = QSUB_THREADS / 32;
-constexpr int QSUB_MAX_ROWS = (QUOKA_MAX_CHUNK + QSUB_CS - 1) / QSUB_CS;
+constexpr int QSUB_MAX_ROWS = (QUOKA_MAX_CHUNK + QSUB_MAX_CS - 1) / QSUB_MAX_CS;   // chunk positions per CTA
 constexpr int QSUB_LPR = 8;                   // lanes per query row
 constexpr int QSUB_RPS = 32 / QSUB_LPR;       // rows per warp step
 constexpr int QSUB_PULL = (QUOKA_MAX_CHUNK + QSUB_THREADS - 1) / QSUB_THREADS;   // keys pulled per thread
@@ -72,8 +75,8 @@ __device__ __forceinline__ float group8_sum(float v) {   // sum over the 8 lanes
   return v;
 }
 
-template <typename T, int D>
-__global__ void __cluster_dims__(QSUB_CS, 1, 1) __launch_bounds__(QSUB_THREADS, 2)
+template <typename T, int D, int CS>
+__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(QSUB_THREADS, 2)
 qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
             int32_t* __restrict__ kept_out, T* __restrict__ qsel, float* __restrict__ qinv,
             float* __restrict__ qbias) {
@@ -91,10 +94,10 @@ qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
   extern __shared__ uint32_t keys[];          // C entries: c_t keys at chunk position t
 
   const int rank = (int)cluster.block_rank();
-  const int bh = blockIdx.x / QSUB_CS;        // b * h_q + h
+  const int bh = blockIdx.x / CS;             // b * h_q + h
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 3, l8 = lane & 7;
-  const int S = (C + QSUB_CS - 1) / QSUB_CS;
+  const int S = (C + CS - 1) / CS;            // <= QSUB_MAX_ROWS (the call picks CS so)
   const int lo = min(C, rank * S), hi = min(C, lo + S);
   const int n = hi - lo;
   const T* qh = q + (size_t)bh * C * D;
@@ -167,7 +170,7 @@ qsub_kernel(const T* __restrict__ q, int C, int nk, int nkp, int nq,
   if (tid < D) {
     float s = 0.f;
 #pragma unroll
-    for (int r = 0; r < QSUB_CS; ++r) s += cluster.map_shared_rank(cta_sum, r)[tid];
+    for (int r = 0; r < CS; ++r) s += cluster.map_shared_rank(cta_sum, r)[tid];
     mdir[tid] = s;
   }
   cluster_arrive();                            // remote reads of cta_sum done; waited below

@@ -394,11 +394,26 @@ quoka_status launch_select(const Dims& d, const SeqTable& tab, long long rows, c
     return launch_topk(d, tab, b_max, idx_out, w, pooled, st);
   }
 
+  // CTAs per query head: the fewest that cover the chunk, doubled while every head's
+  // cluster still fits the SMs at once (two CTAs per SM)
+  int cs = 1;
+  while (cs < QSUB_MAX_CS && (d.C + cs - 1) / cs > QSUB_MAX_ROWS) cs *= 2;
+  while (cs < QSUB_MAX_CS && (long long)d.batch * d.h_q * cs * 2 <= 2LL * sm_count()) cs *= 2;
   const int qs_smem = d.C * 4;                 // the chunk-wide key array
-  if ((e = ensure_smem(qsub_kernel<T, D>, qs_smem)) != cudaSuccess) return cuda_fail(e, "qsub smem");
-  qsub_kernel<T, D><<<d.batch * d.h_q * QSUB_CS, QSUB_THREADS, qs_smem, st>>>(
-      reinterpret_cast<const T*>(q), d.C, w.nk, w.nkp, nq, kept_out, qsel, qinv, qbias);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "qsub launch");
+  auto qsub_launch = [&](auto kern, int csz) -> cudaError_t {
+    cudaError_t err = ensure_smem(kern, qs_smem);
+    if (err != cudaSuccess) return err;
+    kern<<<d.batch * d.h_q * csz, QSUB_THREADS, qs_smem, st>>>(
+        reinterpret_cast<const T*>(q), d.C, w.nk, w.nkp, nq, kept_out, qsel, qinv, qbias);
+    return cudaGetLastError();
+  };
+  switch (cs) {
+    case 1: e = qsub_launch(qsub_kernel<T, D, 1>, 1); break;
+    case 2: e = qsub_launch(qsub_kernel<T, D, 2>, 2); break;
+    case 4: e = qsub_launch(qsub_kernel<T, D, 4>, 4); break;
+    default: e = qsub_launch(qsub_kernel<T, D, 8>, 8); break;
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "qsub launch");
   prof_mark(st, "qsub_kernel");
 
   if (tab.max_prefix > 0) {
