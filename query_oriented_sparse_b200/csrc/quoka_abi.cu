@@ -300,13 +300,28 @@ quoka_status launch_topk(const Dims& d, const SeqTable& tab, int b_max, int32_t*
     prof_mark(st, "topk_block_kernel");
     return QUOKA_OK;
   }
-  const int tk_keys = std::min((tab.max_prefix + TOPK_CS - 1) / TOPK_CS, TOPK_STAGE_KEYS);
+  // CTAs per row: 16, halved (down to 4) while the rows' clusters would not all fit the
+  // SMs at once (one CTA per SM) and a CTA's slice still fits its staging area
+  int cs = TOPK_MAX_CS;
+  while (cs > 4 && (long long)nrows * cs > (long long)sm_count() &&
+         (tab.max_prefix + cs / 2 - 1) / (cs / 2) <= TOPK_STAGE_KEYS)
+    cs /= 2;
+  const int tk_keys = std::min((tab.max_prefix + cs - 1) / cs, TOPK_STAGE_KEYS);
   const int tk_smem = tk_keys * 4;
-  if ((e = ensure_smem(topk_kernel, tk_smem)) != cudaSuccess) return cuda_fail(e, "topk smem");
-  if ((e = ensure_cluster16(topk_kernel)) != cudaSuccess) return cuda_fail(e, "topk cluster size");
-  topk_kernel<<<nrows * TOPK_CS, TOPK_THREADS, tk_smem, st>>>(
-      pooled, w.pooled_stride, w.ncg, w.cg_stride, 1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "topk launch");
+  auto topk_launch = [&](auto kern, int csz) -> cudaError_t {
+    cudaError_t err = ensure_smem(kern, tk_smem);
+    if (err == cudaSuccess && csz > 8) err = ensure_cluster16(kern);
+    if (err != cudaSuccess) return err;
+    kern<<<nrows * csz, TOPK_THREADS, tk_smem, st>>>(
+        pooled, w.pooled_stride, w.ncg, w.cg_stride, 1.0f / (float)d.G, tab, d.h_kv, b_max, idx_out);
+    return cudaGetLastError();
+  };
+  switch (cs) {
+    case 4: e = topk_launch(topk_kernel<4>, 4); break;
+    case 8: e = topk_launch(topk_kernel<8>, 8); break;
+    default: e = topk_launch(topk_kernel<16>, 16); break;
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "topk launch");
   prof_mark(st, "topk_kernel");
   return QUOKA_OK;
 }

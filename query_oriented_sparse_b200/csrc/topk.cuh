@@ -2,8 +2,12 @@
 // ascending index order (QUOKA page, Figure 1(a): the KV cache is sub-selected into a
 // compacted cache before dense attention).
 //
-// One thread-block cluster of TOPK_CS = 16 CTAs per (sequence, KV head); CTA r owns a
-// contiguous slice of the prefix.  The exact B-th largest score is found by a cluster
+// One thread-block cluster of CS CTAs per (sequence, KV head); CTA r owns a contiguous
+// slice of the prefix.  CS is 16 (a non-portable cluster size, opted into at launch) unless
+// the rows' clusters would not all fit the SMs at once (one CTA per SM: 73 registers per
+// thread): then it halves, down to 4, while a CTA's slice still fits its staging area, so
+// many rows run in one wave of clusters instead of several, each wave paying the whole
+// radix select's latency.  The exact B-th largest score is found by a cluster
 // radix select over orderable score keys and the kept indices are emitted in index
 // order (cluster_select.cuh), so the result is deterministic and sorted without a sort.
 // Each CTA first stages its slice's keys in shared memory (coalesced, sixteen loads in
@@ -16,13 +20,13 @@
 
 namespace quoka {
 
-constexpr int TOPK_CS = 16;                   // CTAs per (sequence, KV head); a non-portable
-                                              // cluster size, opted into at launch
+constexpr int TOPK_MAX_CS = 16;               // CTAs per (sequence, KV head) at most
 constexpr int TOPK_THREADS = 512;
 constexpr int TOPK_STAGE_KEYS = 49152;         // keys staged per CTA (192 KB)
 constexpr int TOPK_STAGE_UNROLL = 16;          // staging loads in flight per thread
 
-__global__ void __cluster_dims__(TOPK_CS, 1, 1) __launch_bounds__(TOPK_THREADS)
+template <int CS>
+__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(TOPK_THREADS)
 topk_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, long long cg_stride,
             float inv_G, const __grid_constant__ SeqTable tab, int h_kv, int b_max,
             int32_t* __restrict__ idx_out) {
@@ -31,12 +35,12 @@ topk_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, long l
   extern __shared__ uint32_t staged[];         // TOPK_STAGE_KEYS entries when used
 
   const int rank = (int)cluster.block_rank();
-  const int head = blockIdx.x / TOPK_CS;       // b * h_kv + g
+  const int head = blockIdx.x / CS;            // b * h_kv + g
   const int b = head / h_kv;
   const int P = tab.prefix[b], B = tab.nsel[b];
   int32_t* out = idx_out + (size_t)head * b_max;
   float* sc = pooled + (size_t)head * pooled_stride;
-  const int stride = TOPK_CS * blockDim.x;
+  const int stride = CS * blockDim.x;
 
   if (ncg > 1) {                               // sum the column groups' partial scores
     for (int j = rank * blockDim.x + threadIdx.x; j < P; j += stride) {
@@ -55,7 +59,7 @@ topk_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, long l
   }
   if (B == 0) return;
 
-  const int S = (P + TOPK_CS - 1) / TOPK_CS;
+  const int S = (P + CS - 1) / CS;
   const int lo = min(P, rank * S), hi = min(P, lo + S);
   auto emit = [&](int pos, int j) {
     if (pos < B) out[pos] = j;
@@ -77,11 +81,11 @@ topk_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, long l
     }
     __syncthreads();
     auto key_at = [&](int j) { return staged[j - lo]; };
-    const SelectThreshold th = cluster_threshold<TOPK_CS, true>(cluster, sm, key_at, lo, hi, B);
+    const SelectThreshold th = cluster_threshold<CS, true>(cluster, sm, key_at, lo, hi, B);
     ordered_emit<true>(sm, key_at, lo, hi, th, emit);
   } else {
     auto key_at = [sc](int j) { return float_to_ordered(sc[j]); };
-    const SelectThreshold th = cluster_threshold<TOPK_CS, true>(cluster, sm, key_at, lo, hi, B);
+    const SelectThreshold th = cluster_threshold<CS, true>(cluster, sm, key_at, lo, hi, B);
     ordered_emit<true>(sm, key_at, lo, hi, th, emit);
   }
   cluster_wait();                              // peers' last reads of this CTA's histograms
