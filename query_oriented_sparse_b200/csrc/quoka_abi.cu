@@ -291,7 +291,10 @@ quoka_status launch_topk(const Dims& d, const SeqTable& tab, int b_max, int32_t*
                          const WsLayout& w, float* pooled, cudaStream_t st) {
   cudaError_t e;
   const int nrows = d.batch * d.h_kv;
-  if (tab.max_prefix <= TOPK_BLOCK_MAX_KEYS && nrows >= TOPK_BLOCK_MIN_ROWS) {
+  // one CTA per row when the rows are many, or so short that a cluster's barriers cost
+  // more than it spreads
+  if (tab.max_prefix <= TOPK_BLOCK_MAX_KEYS &&
+      (nrows >= TOPK_BLOCK_MIN_ROWS || tab.max_prefix <= TOPK_BLOCK_ANY_KEYS)) {
     const int smem = std::max(tab.max_prefix, 1) * 4;
     if ((e = ensure_smem(topk_block_kernel, smem)) != cudaSuccess) return cuda_fail(e, "topk_block smem");
     topk_block_kernel<<<nrows, 512, smem, st>>>(pooled, w.pooled_stride, w.ncg, w.cg_stride,

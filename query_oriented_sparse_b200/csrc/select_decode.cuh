@@ -16,7 +16,10 @@
 //                        queries, mean over the group's heads);
 //   topk_block_kernel    one CTA per (sequence, KV head) for rows short enough to stage
 //                        in shared memory: the radix select and the ordered emit of
-//                        cluster_select.cuh with block barriers only.
+//                        cluster_select.cuh with block barriers only.  Taken when there
+//                        are at least 32 rows of at most 32768 keys, or rows of at most
+//                        8192 keys however few (gqa_8k's 8 rows of 8192: 19.4 us against
+//                        23.5 us for 16-CTA clusters).
 #pragma once
 #include "cluster_select.cuh"
 #include "tc_ptx.cuh"
@@ -30,6 +33,7 @@ constexpr int SCD_BATCHES = 8;                              // 32-key batches pe
 constexpr int SCD_KEYS = SCD_WARPS * SCD_BATCHES * 32;      // keys per CTA
 constexpr int TOPK_BLOCK_MAX_KEYS = 32768;                  // staged keys (128 KB)
 constexpr int TOPK_BLOCK_MIN_ROWS = 32;                     // (sequence, KV head) rows
+constexpr int TOPK_BLOCK_ANY_KEYS = 8192;                   // rows this short, however few
 
 __global__ void kept_all_kernel(int32_t* __restrict__ kept_out, int heads, int C, int nq) {
   const long long n = (long long)heads * nq;

@@ -13,8 +13,8 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("kind", ["chunk", "decode", "f32"])
 def test_kernel_timer_names_every_launch(kind, cuda_device):
     if kind == "chunk":
-        w = W.custom("prof_chunk", h_q=8, h_kv=2, head_dim=128, chunk=256, prefix=3000, nq=32,
-                     budget=512, recipe="rank4", seed=91)
+        w = W.custom("prof_chunk", h_q=8, h_kv=2, head_dim=128, chunk=256, prefix=9000, nq=32,
+                     budget=1024, recipe="rank4", seed=91)
         expect = ["qsub_kernel", "score_tc_kernel", "topk_kernel", "compact_kv_kernel",
                   "attn_tc2_kernel"]
     elif kind == "decode":
@@ -25,7 +25,7 @@ def test_kernel_timer_names_every_launch(kind, cuda_device):
     else:
         w = W.custom("prof_f32", h_q=4, h_kv=1, head_dim=64, chunk=64, prefix=500, nq=8,
                      budget=64, dtype="f32", seed=93)
-        expect = ["qsub_kernel", "score_simt_kernel", "topk_kernel", "attn_simt_kernel"]
+        expect = ["qsub_kernel", "score_simt_kernel", "topk_block_kernel", "attn_simt_kernel"]
     t = W.generate(w)
     dev = cuda_device
     q, k, v = t.q.to(dev), t.k_cache.to(dev), t.v_cache.to(dev)
