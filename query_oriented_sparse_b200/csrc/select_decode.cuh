@@ -201,6 +201,14 @@ topk_block_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, 
   const int P = tab.prefix[b], B = tab.nsel[b];
   int32_t* out = idx_out + (size_t)head * b_max;
   float* sc = pooled + (size_t)head * pooled_stride;
+  if (ncg > 1) {                                           // column groups, in group order
+    for (int j = threadIdx.x; j < P; j += blockDim.x) {
+      float s = sc[j];
+      for (int c = 1; c < ncg; ++c) s += sc[c * cg_stride + j];
+      sc[j] = s * inv_G;
+    }
+    __syncthreads();
+  }
   for (int i = B + threadIdx.x; i < b_max; i += blockDim.x) out[i] = -1;
   if (B >= P) {                                            // every prefix key (P == 0 too)
     for (int i = threadIdx.x; i < P; i += blockDim.x) out[i] = i;
@@ -219,14 +227,7 @@ topk_block_kernel(float* __restrict__ pooled, long long pooled_stride, int ncg, 
 #pragma unroll
     for (int u = 0; u < TOPK_STAGE_UNROLL; ++u) {
       const int j = j0 + u * blockDim.x;
-      if (j >= P) continue;
-      float s = v[u];
-      if (ncg > 1) {                                       // column groups, in group order
-        for (int c = 1; c < ncg; ++c) s += sc[c * cg_stride + j];
-        s *= inv_G;
-        sc[j] = s;
-      }
-      staged[j] = float_to_ordered(s);
+      if (j < P) staged[j] = float_to_ordered(v[u]);
     }
   }
   __syncthreads();

@@ -25,6 +25,11 @@ CASES = [
     # 2 rows of 4000 keys -> one CTA per row
     W.custom("topk_block_few", h_q=8, h_kv=2, head_dim=64, chunk=64, prefix=(4000,), nq=16,
              budget=(600,), seed=804, recipe="rank4"),
+    # one CTA per row with the kept queries in two column groups (16 heads x 64), one
+    # sequence keeping every prefix key and one keeping none: the groups' partial scores
+    # are summed before either early exit
+    W.custom("topk_block_groups_edges", h_q=16, h_kv=1, head_dim=128, chunk=96, prefix=(600, 300),
+             nq=64, budget=(700, 0), seed=809, recipe="rank4"),
     # subselect: 192 heads of 256 queries -> 1 CTA per head
     W.custom("qsub_cs1", h_q=64, h_kv=8, head_dim=128, chunk=256, prefix=(300, 200, 250), nq=32,
              budget=(64, 64, 64), seed=805, recipe="gauss"),
