@@ -24,7 +24,8 @@ namespace quoka {
 
 constexpr int PTC_THREADS = 1024;
 constexpr int PTC_MAX_WORDS = 8192;       // sequence bitmap: up to 262144 rows
-constexpr int PTC_BATCH = 8;              // set entries a lane has in flight
+constexpr int PTC_BATCH = 8;              // set entries a lane has in flight (scalar loads)
+constexpr int PTC_BATCH4 = 8;             // 16-byte loads a lane has in flight (32 entries)
 
 // Shared memory of the union kernel: the sequence bitmap, its word offsets, and one
 // mask row per warp.
@@ -60,6 +61,41 @@ perq_tc_union_kernel(const int32_t* __restrict__ sel, const __grid_constant__ Se
     return head < G && pos < C;
   };
 
+  // every entry of a set row, handed to fn one by one with many loads in flight per lane:
+  // 16-byte loads when the rows are 16-byte aligned (S a multiple of 4), else 4-byte ones
+  auto for_set = [&](const int32_t* srow, auto&& fn) {
+    if ((S & 3) == 0) {
+      const int4* s4 = reinterpret_cast<const int4*>(srow);
+      const int S4 = S >> 2;
+      for (int i0 = 0; i0 < S4; i0 += 32 * PTC_BATCH4) {
+        int4 x[PTC_BATCH4];                                    // all loads in flight first
+#pragma unroll
+        for (int u = 0; u < PTC_BATCH4; ++u) {
+          const int i = i0 + u * 32 + lane;
+          x[u] = i < S4 ? __ldg(s4 + i) : make_int4(-1, -1, -1, -1);
+        }
+#pragma unroll
+        for (int u = 0; u < PTC_BATCH4; ++u) {
+          fn(x[u].x);
+          fn(x[u].y);
+          fn(x[u].z);
+          fn(x[u].w);
+        }
+      }
+    } else {
+      for (int i0 = 0; i0 < S; i0 += 32 * PTC_BATCH) {
+        int x[PTC_BATCH];
+#pragma unroll
+        for (int u = 0; u < PTC_BATCH; ++u) {
+          const int i = i0 + u * 32 + lane;
+          x[u] = i < S ? __ldg(srow + i) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < PTC_BATCH; ++u) fn(x[u]);
+      }
+    }
+  };
+
   for (int w = tid; w < W; w += PTC_THREADS) bm[w] = 0u;
   __syncthreads();
   // a warp per row; a bit already set (most of them, when rows share their keys) costs a
@@ -68,21 +104,12 @@ perq_tc_union_kernel(const int32_t* __restrict__ sel, const __grid_constant__ Se
     int head, pos;
     if (!row_of(rr, head, pos)) continue;
     const int32_t* srow = sel + (((size_t)b * h_q + (size_t)g * G + head) * C + pos) * S;
-    for (int i0 = 0; i0 < S; i0 += 32 * PTC_BATCH) {
-      int x[PTC_BATCH];                                        // all loads in flight first
-#pragma unroll
-      for (int u = 0; u < PTC_BATCH; ++u) {
-        const int i = i0 + u * 32 + lane;
-        x[u] = i < S ? __ldg(srow + i) : -1;
-      }
-#pragma unroll
-      for (int u = 0; u < PTC_BATCH; ++u) {
-        if (x[u] < 0) continue;
-        if (x[u] >= N) { flag_error(ERR_BAD_INDEX); continue; }
-        const uint32_t bit = 1u << (x[u] & 31);
-        if (!(bm[x[u] >> 5] & bit)) atomicOr(&bm[x[u] >> 5], bit);
-      }
-    }
+    for_set(srow, [&](int x) {
+      if (x < 0) return;
+      if (x >= N) { flag_error(ERR_BAD_INDEX); return; }
+      const uint32_t bit = 1u << (x & 31);
+      if (!(bm[x >> 5] & bit)) atomicOr(&bm[x >> 5], bit);
+    });
   }
   __syncthreads();
   // exclusive scan of the words' popcounts (each thread a contiguous run of words)
@@ -141,21 +168,12 @@ perq_tc_union_kernel(const int32_t* __restrict__ sel, const __grid_constant__ Se
     int head, pos;
     if (row_of(rr, head, pos)) {
       const int32_t* srow = sel + (((size_t)b * h_q + (size_t)g * G + head) * C + pos) * S;
-      for (int i0 = 0; i0 < S; i0 += 32 * PTC_BATCH) {
-        int x[PTC_BATCH];
-#pragma unroll
-        for (int u = 0; u < PTC_BATCH; ++u) {
-          const int i = i0 + u * 32 + lane;
-          x[u] = i < S ? __ldg(srow + i) : -1;
-        }
-#pragma unroll
-        for (int u = 0; u < PTC_BATCH; ++u) {
-          if (x[u] < 0 || x[u] >= N) continue;
-          const uint32_t word = bm[x[u] >> 5];
-          const int rank = roff[x[u] >> 5] + __popc(word & ((1u << (x[u] & 31)) - 1u));
-          if (rank < nu) atomicOr(&my[rank >> 5], 1u << (rank & 31));
-        }
-      }
+      for_set(srow, [&](int x) {
+        if (x < 0 || x >= N) return;
+        const uint32_t word = bm[x >> 5];
+        const int rank = roff[x >> 5] + __popc(word & ((1u << (x & 31)) - 1u));
+        if (rank < nu) atomicOr(&my[rank >> 5], 1u << (rank & 31));
+      });
     }
     __syncwarp();
     uint32_t* dst = mask + (tile * 256 + rr) * (size_t)mwords;

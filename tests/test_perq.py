@@ -99,6 +99,9 @@ TC_CASES = [
         seed=83), 64, 128, 0.95, False),
     (C_("pqtc_g16", h_q=32, h_kv=2, head_dim=128, chunk=20, prefix=2500, nq=1, budget=1,
         seed=84), 32, 16, 0.9, True),
+    # a set size that is not a multiple of 4: the union kernel's 4-byte entry loads
+    (C_("pqtc_g2_s37", h_q=4, h_kv=2, head_dim=128, chunk=70, prefix=1800, nq=1, budget=1,
+        seed=85), 37, 32, 0.8, False),
 ]
 
 
