@@ -81,8 +81,8 @@ def test_stage_model_ctx_128k():
 def test_attn_traffic_is_pinned_to_workload():
     assert bench.attn_traffic(W.WORKLOADS["gqa_8k"]) is None
     t = bench.attn_traffic(W.WORKLOADS["ctx_128k"])
-    # one ncu capture of the kernel on this workload: dram read 117.53 MB + write 16.55 MB
-    assert t is None or abs(t - 134.08e6) < 1e5
+    # one ncu capture of the kernel on this workload: dram read 117.63 MB + write 19.44 MB
+    assert t is None or abs(t - 137.07e6) < 1e5
 
 
 def test_oracle_prompt_sample_extrapolates():
